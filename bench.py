@@ -1,0 +1,452 @@
+#!/usr/bin/env python3
+"""CSA2 decode benchmark: 40-layer decode step, batch 16, 131,072-token context.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 2]
+
+One step = one CSA2 decode step of every layer of the workload (window append,
+source cache write, every Full/Reindex scan + Top-K, every layer's attention)
+for the whole batch, through the C ABI's csa2_layer_step, replayed from a CUDA
+graph.  Metric: layer-steps/s (one layer x one decode step for the batch).
+Multi-GPU: one process per GPU, each with its own batch (the path shards by
+sequence, no collective): weak scaling, value = all ranks' layer-steps / max time.
+
+``--impl reference`` times the CPU oracle (the plain C reference) on the host
+cores on a bounded sample of the same workload; it prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode layer-steps/s at 128K ctx"
+UNIT = "layer-steps/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.samples = []  # (t, sm, smax, reasons set)
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, smax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            reasons = {n for n, v in zip(names, parts[5:9]) if v.lower() == "active"}
+            self.samples.append((time.time(), sm, smax, reasons))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        where = "timed"
+        if len(win) < 3:
+            win = [s for s in self.samples if s[0] <= t1]
+            where = "warmup+timed"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": "none"}
+        reasons = sorted(set().union(*[s[3] for s in win]))
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": max(s[2] for s in win),
+                "reasons": reasons, "samples": len(win), "window": where}
+
+
+# ---------------------------------------------------------------- helpers
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def scan_traffic(kernel_file: str):
+    """Per-launch DRAM bytes of the scan from a committed ncu summary, only while
+    the kernel source is unchanged since the capture (else None)."""
+    p = os.path.join(ROOT, "profiles", "scan_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        with open(kernel_file, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        if d.get("source_sha") != sha:
+            return None, d
+        return d, d
+    except (OSError, ValueError):
+        return None, None
+
+
+def step_bytes(wl, n_entries):
+    """Algorithmic HBM bytes of one decode step (our accounting of the path):
+    every scan reads its source's keys (68 B/entry) and its query; every
+    attention reads K entries (288 B) + indices and the 128-token window and
+    its query; outputs fp32; the cache write of the completed groups."""
+    t = wl.table
+    B, H, Hi, K = wl.B, wl.H, wl.H_idx, wl.K
+    rd = wr = 0
+    scan_rd = 0
+    for l in t.scan_layers():
+        n = sum(n_entries[t.src[l]])
+        scan_rd += n * 68 + B * (Hi * 128 * 2 + Hi * 4)
+        wr += B * K * 4
+    rd += scan_rd
+    for l, m in enumerate(t.mode):
+        rd += B * (WIN * 512 * 2 + H * 512 * 2)
+        if m != 0:
+            rd += B * K * (288 + 4)
+        wr += B * H * 512 * 4
+    return rd, wr, scan_rd
+
+
+WIN = 128
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(wl, seqs=(0,), layers=None, budget_s=None):
+    """Time the oracle on `layers` for `seqs` (caches built untimed).  Returns
+    (seconds per (scan layer, sequence), seconds per (attention-only layer,
+    sequence), threads, description)."""
+    import numpy as np
+    import oracle
+    from fp4_sparse_attention_pack_b200 import workloads as W
+    from tests.oracle_models import ref_cache, ref_window
+    t = wl.table
+    layers = layers if layers is not None else list(range(2, 8))
+    srcs = sorted({t.src[l] for l in layers if t.mode[l] != W.SWA_ONLY})
+    caches = {s: ref_cache(wl, s, list(seqs), wl.T, cap=wl.T // t.ratios[s] + 64) for s in srcs}
+    t_scan, t_attn = [], []
+    for i, b in enumerate(seqs):
+        idx = {}
+        for l in layers:
+            m = t.mode[l]
+            ring, cnt = ref_window(wl, l, b, wl.T)
+            t0 = time.perf_counter()
+            if m in (W.FULL, W.REINDEX):
+                c = caches[t.src[l]]
+                sc = c.scores(i, W.query_idx(wl, l, 0)[b], W.head_weights(wl, l, 0)[b])
+                idx[l] = oracle.topk(sc, wl.K)
+            sel = idx.get(l if m != W.REUSE else t.idx_src[l])
+            if m == W.SWA_ONLY:
+                items = oracle.attention_items(np.zeros((1, 256), np.uint8), np.zeros((1, 32), np.uint8),
+                                               0, np.zeros(0, np.int32), ring, min(cnt, WIN))
+            else:
+                c = caches[t.src[l]]
+                items = oracle.attention_items(c.mc[i], c.ms[i], int(c.n[i]), sel, ring, min(cnt, WIN))
+            oracle.attention(W.query(wl, l, 0)[b], items, wl.scale)
+            dt = time.perf_counter() - t0
+            (t_scan if m in (W.FULL, W.REINDEX) else t_attn).append(dt)
+    desc = (f"oracle on layers {layers[0]}-{layers[-1]} x sequences {list(seqs)} of the 40-layer "
+            f"step (Top-K scan over {wl.T // 2} entries, 64 heads, attention over K + 128 items); "
+            f"per-layer-step time = 16 x (23 scan-layer + 17 attention-only-layer) sequence times")
+    return (statistics.mean(t_scan) if t_scan else 0.0, statistics.mean(t_attn) if t_attn else 0.0,
+            oracle.threads(), desc)
+
+
+def cpu_baseline(wl):
+    ts, ta, thr, desc = oracle_sample(wl)
+    n_scan = len(wl.table.scan_layers())
+    n_attn = wl.table.n_layers - n_scan
+    step_s = wl.B * (n_scan * ts + n_attn * ta)
+    return {"value": wl.table.n_layers / step_s, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": desc}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank):
+    import numpy as np
+    from fp4_sparse_attention_pack_b200 import workloads as W
+    import oracle
+    from tests.oracle_models import ref_cache, ref_window
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.config]
+    t = wl.table
+    # untimed set-up: the oracle packs one sequence of every source
+    caches = {s: ref_cache(wl, s, [0], wl.T, cap=wl.T // t.ratios[s] + 64) for s in range(t.n_sources)}
+    rings = {l: ref_window(wl, l, 0, wl.T) for l in range(t.n_layers)}
+    idx = {}
+
+    def one(i):
+        l = i % t.n_layers
+        m = t.mode[l]
+        if m in (W.FULL, W.REINDEX):
+            c = caches[t.src[l]]
+            idx[l] = oracle.topk(c.scores(0, W.query_idx(wl, l, 0)[0], W.head_weights(wl, l, 0)[0]), wl.K)
+        ring, cnt = rings[l]
+        if m == W.SWA_ONLY:
+            items = oracle.attention_items(np.zeros((1, 256), np.uint8), np.zeros((1, 32), np.uint8), 0,
+                                           np.zeros(0, np.int32), ring, min(cnt, WIN))
+        else:
+            c = caches[t.src[l]]
+            sel = idx.get(l if m != W.REUSE else t.idx_src[l])
+            if sel is None:  # a Reuse layer whose source was not run in this window
+                src = t.idx_src[l]
+                cs = caches[t.src[src]]
+                sel = idx[src] = oracle.topk(cs.scores(0, W.query_idx(wl, src, 0)[0],
+                                                       W.head_weights(wl, src, 0)[0]), wl.K)
+            items = oracle.attention_items(c.mc[0], c.ms[0], int(c.n[0]), sel, ring, min(cnt, WIN))
+        oracle.attention(W.query(wl, l, 0)[0], items, wl.scale)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(args.warmup + i)
+    dt = time.perf_counter() - t0
+    # each sample step is one layer for one of the batch's sequences: 1/B layer-step
+    value = (args.steps / wl.B) / dt
+    desc = (f"each step: the oracle on one layer (cycling through the 40-layer schedule) for one of the "
+            f"{wl.B} sequences; value = (steps / {wl.B}) / seconds")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.T, "layers": t.n_layers},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import ctypes
+    import torch
+    import torch.distributed as dist
+    import fp4_sparse_attention_pack_b200 as csa
+    from fp4_sparse_attention_pack_b200 import engine, workloads as W
+
+    torch.cuda.set_device(local_rank)
+    dev = f"cuda:{local_rank}"
+    base = W.WORKLOADS[args.config]
+    wl = W.small(base, seed=base.seed + 1000 * rank)  # each rank: its own batch of sequences
+    extra = args.warmup + args.steps + 2 * args.profile_steps + 8
+    dm = engine.DecodeModel(wl, dev, steps_capacity=extra)
+    dm.fill()
+    dm.gen_step_inputs(0)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    stream = torch.cuda.Stream()
+    torch.cuda.current_stream().wait_stream(torch.cuda.default_stream())
+    # one eager step (also validates arguments), then capture
+    with torch.cuda.stream(stream):
+        dm.step(stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        dm.step(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    time.sleep(0.25)
+    clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    n_ent = [dm.caches[s].n_entries.cpu().tolist() for s in range(dm.S)]
+    status = dm.status_bits()
+
+    # per-phase device times of the same step (eager launches with events)
+    names = ["window_append", "cache_write", "query_quant", "index_scan", "topk", "attention",
+             "attn_combine"]
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(8 * args.profile_steps)]
+    lib = csa.lib()
+    lib.csa2_layer_step_profiled.restype = ctypes.c_int
+    lib.csa2_layer_step_profiled.argtypes = [ctypes.POINTER(csa.csa2_model), ctypes.POINTER(csa.csa2_step_in),
+                                             ctypes.POINTER(csa.csa2_step_out), ctypes.c_void_p,
+                                             ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
+    phase = [[] for _ in names]
+    with torch.cuda.stream(stream):
+        for i in range(args.profile_steps):
+            e = evs[8 * i:8 * i + 8]
+            arr = (ctypes.c_void_p * 8)(*[x.cuda_event for x in e])
+            rc = lib.csa2_layer_step_profiled(ctypes.byref(dm.model), ctypes.byref(dm._in),
+                                              ctypes.byref(dm._out), dm.ws.data_ptr(),
+                                              dm.ws.numel(), stream.cuda_stream, arr)
+            if rc != 0:
+                raise csa.Csa2Error(rc, "csa2_layer_step_profiled")
+    torch.cuda.synchronize()
+    for i in range(args.profile_steps):
+        e = evs[8 * i:8 * i + 8]
+        for k in range(7):
+            phase[k].append(e[k].elapsed_time(e[k + 1]))
+    phase_ms = {n: statistics.mean(v) for n, v in zip(names, phase)}
+
+    # end to end: pinned host inputs -> step -> host outputs, every step
+    e2e = None
+    h2d = d2h = 0
+    ins = [dm.x_new, dm.g_new, dm.q, dm.q_idx, dm.w, dm.win_tok]
+    outs = [dm.out, dm.idx]
+    host_in = [t.cpu().pin_memory() for t in ins]
+    host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in ins)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    e2e_steps = max(3, min(args.steps, 30))
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            for d, h in zip(ins, host_in):
+                d.copy_(h, non_blocking=True)
+            dm.step(stream)
+            for d, h in zip(outs, host_out):
+                h.copy_(d, non_blocking=True)
+        f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    barrier()
+    if rank != 0:
+        return
+
+    L = wl.table.n_layers
+    value = L * world / (ms / 1e3)
+    rd, wr, scan_rd = step_bytes(wl, n_ent)
+    peak, peak_kind = measured_peaks()
+    scan_ms = phase_ms["index_scan"]
+    achieved = scan_rd / (scan_ms / 1e3) / 1e9
+    tr, _ = scan_traffic(os.path.join(ROOT, "fp4_sparse_attention_pack_b200", "csrc", "scan.cu"))
+    traffic = tr["bytes_per_launch_at_workload"] if tr else None
+    launches_per_step = 1 + 2 * dm.S + 3 + 2
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.T,
+                   "layers": L, "scans_per_step": len(wl.table.scan_layers()), "H": wl.H,
+                   "H_idx": wl.H_idx, "top_k": wl.K, "parallelism": f"dp{world} (replicas, no collective)",
+                   "cache_format": "E2M1+E4M3/16 main, MXFP4 indexer keys",
+                   "l2": "inputs larger than L2: %.2f GB read per step" % (rd / 1e9),
+                   "cuda_graph": True},
+        "hbm": {"step_read_bytes": rd, "step_write_bytes": wr,
+                "achieved_gbs": (rd + wr) / (ms / 1e3) / 1e9,
+                "frac_of_8tbs": (rd + wr) / (ms / 1e3) / 8e12,
+                "frac_of_measured": (rd + wr) / (ms / 1e3) / (peak * 1e9)},
+        "roofline": {"kernel": "index_scan", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": peak_kind, "algorithmic_bytes_per_launch": scan_rd,
+                     "launch_ms": scan_ms},
+        "phase_ms": phase_ms,
+        "e2e": {"value": L * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(W.WORKLOADS[args.config])
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,379 @@
+// C ABI of the CSA2 library: argument validation, workspace layout and the
+// per-step schedule of the Full / Reindex / Reuse mode table ("Résumé
+// exécutif", CSA2 table: Full computes cache, keys and indices; Reindex reuses
+// cache and keys and recomputes indices; Reuse reuses all three).
+//
+// Everything is validated before the first launch, so an error return means
+// nothing was enqueued.  Nothing is allocated and nothing synchronises, so
+// every entry point can be captured in a CUDA graph.
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace csa2;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cache(const csa2_cache* c) {
+    if (!c) return CSA2_ERR_INVALID_ARG;
+    if (!c->main_codes || !c->main_scales || !c->idx_codes || !c->idx_scales || !c->page_table ||
+        !c->n_entries || !c->pend_x || !c->pend_g || !c->pend_valid || !c->status)
+        return CSA2_ERR_INVALID_ARG;
+    if (c->batch < 1 || c->max_pages < 1 || c->num_pages < 1 || (c->ratio != 1 && c->ratio != 2))
+        return CSA2_ERR_INVALID_ARG;
+    if ((int64_t)c->max_pages * PAGE > (int64_t)1 << 30) return CSA2_ERR_UNSUPPORTED;
+    if (!a16(c->main_codes) || !a16(c->main_scales) || !a16(c->idx_codes) || !a16(c->idx_scales) ||
+        !a16(c->page_table) || !a16(c->n_entries) || !a16(c->pend_x) || !a16(c->pend_g) ||
+        !a16(c->pend_valid) || !a16(c->status))
+        return CSA2_ERR_ALIGN;
+    return CSA2_OK;
+}
+
+int check_window(const csa2_window* w, int batch) {
+    if (!w || !w->tokens || !w->count || w->batch != batch) return CSA2_ERR_INVALID_ARG;
+    if (!a16(w->tokens) || !a16(w->count)) return CSA2_ERR_ALIGN;
+    return CSA2_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
+
+size_t topk_ws_one(int batch, int max_entries, int H_idx) {
+    return align_up((size_t)batch * H_idx * ICB) + align_up((size_t)batch * H_idx * ISB) +
+           align_up((size_t)batch * max_entries * sizeof(float));
+}
+
+// Carve one scan problem's scratch out of ws.
+void carve_scan(ScanProblem& P, uint8_t* ws, int batch, int max_entries, int H_idx) {
+    P.qc = ws;
+    ws += align_up((size_t)batch * H_idx * ICB);
+    P.qs = ws;
+    ws += align_up((size_t)batch * H_idx * ISB);
+    P.scores = reinterpret_cast<float*>(ws);
+    P.score_stride = max_entries;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa2_version(void) { return (0 << 16) | 1; }
+
+const char* csa2_strerror(int status) {
+    switch (status) {
+        case CSA2_OK: return "ok";
+        case CSA2_ERR_INVALID_ARG: return "invalid argument";
+        case CSA2_ERR_ALIGN: return "device pointer not 16-byte aligned";
+        case CSA2_ERR_UNSUPPORTED: return "size not supported by this build";
+        case CSA2_ERR_CUDA: return "CUDA launch or runtime error";
+        case CSA2_ERR_TIMEOUT: return "bounded device wait timed out";
+        case CSA2_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int csa2_pack_cache(const csa2_cache* cache, const void* x, int x_dtype, const float* gates,
+                    const float* w_idx, int T_new, csa2_stream stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (T_new < 0 || (x_dtype != CSA2_DTYPE_BF16 && x_dtype != CSA2_DTYPE_F32))
+        return CSA2_ERR_INVALID_ARG;
+    if (T_new == 0) return CSA2_OK;
+    if (!x || !gates || !w_idx) return CSA2_ERR_INVALID_ARG;
+    if (!a16(x) || !a16(w_idx)) return CSA2_ERR_ALIGN;
+    if ((int64_t)T_new > (int64_t)cache->max_pages * PAGE * 2) return CSA2_ERR_INVALID_ARG;
+    return cuda_status(launch_pack(view_of(*cache), x, x_dtype == CSA2_DTYPE_F32, gates, w_idx, T_new,
+                                   (cudaStream_t)stream));
+}
+
+size_t csa2_index_topk_workspace(int batch, int max_entries, int H_idx, int K) {
+    (void)K;
+    if (batch < 1 || max_entries < 0 || H_idx < 1) return 0;
+    return topk_ws_one(batch, max_entries, H_idx);
+}
+
+int csa2_index_topk(const csa2_cache* cache, const uint16_t* q_idx, const float* w, int H_idx, int K,
+                    int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
+                    csa2_stream stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (H_idx < 1 || H_idx > CSA2_MAX_H_IDX || K < 1 || K > CSA2_MAX_K) return CSA2_ERR_INVALID_ARG;
+    if (!q_idx || !w || !idx_out) return CSA2_ERR_INVALID_ARG;
+    if (!a16(q_idx) || !a16(w) || !a16(idx_out) || (score_out && !a16(score_out)) || (ws && !a16(ws)))
+        return CSA2_ERR_ALIGN;
+    const int cap = cache->max_pages * PAGE;
+    const size_t need = topk_ws_one(cache->batch, cap, H_idx);
+    if (!ws || ws_bytes < need) return CSA2_ERR_WORKSPACE;
+    ScanBatch sb;
+    std::memset(&sb, 0, sizeof(sb));
+    sb.n = 1;
+    sb.H_idx = H_idx;
+    sb.K = K;
+    ScanProblem& P = sb.p[0];
+    P.cache = view_of(*cache);
+    P.q_idx = q_idx;
+    P.w = w;
+    P.idx_out = idx_out;
+    P.score_out = score_out;
+    carve_scan(P, static_cast<uint8_t*>(ws), cache->batch, cap, H_idx);
+    return cuda_status(launch_index_topk(sb, (cudaStream_t)stream));
+}
+
+size_t csa2_sparse_attn_workspace(int batch, int H, int K) {
+    if (batch < 1 || H < 1 || K < 0) return 0;
+    return attn_workspace_bytes(1, batch, H, K);
+}
+
+int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const int32_t* idx, int K,
+                     const csa2_window* win, float scale, float* out, void* ws, size_t ws_bytes,
+                     csa2_stream stream) {
+    if (H < 1 || H > CSA2_MAX_H || K < 0 || K > CSA2_MAX_K || !q || !out || !win)
+        return CSA2_ERR_INVALID_ARG;
+    int batch = win->batch;
+    if (K > 0) {
+        int rc = check_cache(cache);
+        if (rc) return rc;
+        if (!idx) return CSA2_ERR_INVALID_ARG;
+        if (!a16(idx)) return CSA2_ERR_ALIGN;
+        if (cache->batch != batch) return CSA2_ERR_INVALID_ARG;
+    }
+    int rc = check_window(win, batch);
+    if (rc) return rc;
+    if (batch < 1) return CSA2_ERR_INVALID_ARG;
+    if (!a16(q) || !a16(out) || (ws && !a16(ws))) return CSA2_ERR_ALIGN;
+    const size_t need = attn_workspace_bytes(1, batch, H, K);
+    if (!ws || ws_bytes < need) return CSA2_ERR_WORKSPACE;
+    AttnBatch ab;
+    std::memset(&ab, 0, sizeof(ab));
+    ab.n = 1;
+    ab.batch = batch;
+    ab.H = H;
+    ab.Kmax = K;
+    ab.scale = scale;
+    const size_t units = need / ((D + 2) * sizeof(float));
+    ab.part_o = static_cast<float*>(ws);
+    ab.part_ml = ab.part_o + units * D;
+    AttnProblem& P = ab.p[0];
+    if (K > 0) P.cache = view_of(*cache);
+    P.q = q;
+    P.idx = idx;
+    P.win = win->tokens;
+    P.win_count = win->count;
+    P.out = out;
+    P.K = K;
+    return cuda_status(launch_sparse_attn(ab, (cudaStream_t)stream));
+}
+
+int csa2_window_append(const csa2_window* win, const uint16_t* tok, csa2_stream stream) {
+    if (!win || !tok) return CSA2_ERR_INVALID_ARG;
+    int rc = check_window(win, win->batch);
+    if (rc) return rc;
+    if (win->batch < 1) return CSA2_ERR_INVALID_ARG;
+    if (!a16(tok)) return CSA2_ERR_ALIGN;
+    WinAppend wa;
+    std::memset(&wa, 0, sizeof(wa));
+    wa.n = 1;
+    wa.batch = win->batch;
+    wa.tokens[0] = win->tokens;
+    wa.count[0] = win->count;
+    wa.tok[0] = tok;
+    return cuda_status(launch_window_append(wa, (cudaStream_t)stream));
+}
+
+// ---------------------------------------------------------------- layer step
+
+namespace {
+
+int check_model(const csa2_model* m) {
+    if (!m || m->n_layers < 1 || m->n_layers > CSA2_MAX_LAYERS || m->n_sources < 1 ||
+        m->n_sources > CSA2_MAX_SOURCES || !m->mode || !m->src || !m->idx_src || !m->caches ||
+        !m->w_idx || !m->windows)
+        return CSA2_ERR_INVALID_ARG;
+    if (m->batch < 1 || m->H < 1 || m->H > CSA2_MAX_H || m->H_idx < 1 || m->H_idx > CSA2_MAX_H_IDX ||
+        m->K < 1 || m->K > CSA2_MAX_K)
+        return CSA2_ERR_INVALID_ARG;
+    int full_of[CSA2_MAX_SOURCES];
+    for (int s = 0; s < m->n_sources; ++s) full_of[s] = -1;
+    for (int l = 0; l < m->n_layers; ++l) {
+        const int md = m->mode[l], s = m->src[l];
+        if (md < CSA2_MODE_SWA_ONLY || md > CSA2_MODE_REUSE) return CSA2_ERR_INVALID_ARG;
+        if (md == CSA2_MODE_SWA_ONLY) continue;
+        if (s < 0 || s >= m->n_sources) return CSA2_ERR_INVALID_ARG;
+        if (md == CSA2_MODE_FULL) {
+            if (full_of[s] >= 0 || m->idx_src[l] != l) return CSA2_ERR_INVALID_ARG;
+            full_of[s] = l;
+        } else if (md == CSA2_MODE_REINDEX) {
+            if (full_of[s] < 0 || m->idx_src[l] != l) return CSA2_ERR_INVALID_ARG;
+        } else {
+            const int j = m->idx_src[l];
+            if (j < 0 || j >= l || m->src[j] != s ||
+                (m->mode[j] != CSA2_MODE_FULL && m->mode[j] != CSA2_MODE_REINDEX))
+                return CSA2_ERR_INVALID_ARG;
+        }
+    }
+    for (int s = 0; s < m->n_sources; ++s) {
+        if (full_of[s] < 0) return CSA2_ERR_INVALID_ARG;
+        int rc = check_cache(&m->caches[s]);
+        if (rc) return rc;
+        if (m->caches[s].batch != m->batch || !m->w_idx[s]) return CSA2_ERR_INVALID_ARG;
+        if (!a16(m->w_idx[s])) return CSA2_ERR_ALIGN;
+    }
+    for (int l = 0; l < m->n_layers; ++l) {
+        int rc = check_window(&m->windows[l], m->batch);
+        if (rc) return rc;
+    }
+    return CSA2_OK;
+}
+
+int max_entries(const csa2_model* m) {
+    int cap = 0;
+    for (int s = 0; s < m->n_sources; ++s) cap = std::max(cap, m->caches[s].max_pages * PAGE);
+    return cap;
+}
+
+int n_scans(const csa2_model* m) {
+    int n = 0;
+    for (int l = 0; l < m->n_layers; ++l)
+        n += (m->mode[l] == CSA2_MODE_FULL || m->mode[l] == CSA2_MODE_REINDEX);
+    return n;
+}
+
+}  // namespace
+
+size_t csa2_layer_step_workspace(const csa2_model* m) {
+    if (check_model(m)) return 0;
+    return (size_t)n_scans(m) * topk_ws_one(m->batch, max_entries(m), m->H_idx) +
+           align_up(attn_workspace_bytes(m->n_layers, m->batch, m->H, m->K));
+}
+
+namespace {
+
+int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step_out* out, void* ws,
+                    size_t ws_bytes, csa2_stream stream, cudaEvent_t* ev) {
+    int rc = check_model(m);
+    if (rc) return rc;
+    if (!in || !out || !in->x_new || !in->g_new || !in->q || !in->win_tok || !out->out)
+        return CSA2_ERR_INVALID_ARG;
+    const int L = m->n_layers, B = m->batch;
+    for (int l = 0; l < L; ++l) {
+        if (!in->q[l] || !in->win_tok[l] || !out->out[l]) return CSA2_ERR_INVALID_ARG;
+        if (!a16(in->q[l]) || !a16(in->win_tok[l]) || !a16(out->out[l])) return CSA2_ERR_ALIGN;
+        const int md = m->mode[l];
+        if (md == CSA2_MODE_FULL || md == CSA2_MODE_REINDEX) {
+            if (!in->q_idx || !in->w || !out->idx || !in->q_idx[l] || !in->w[l] || !out->idx[l])
+                return CSA2_ERR_INVALID_ARG;
+            if (!a16(in->q_idx[l]) || !a16(in->w[l]) || !a16(out->idx[l])) return CSA2_ERR_ALIGN;
+        }
+    }
+    for (int s = 0; s < m->n_sources; ++s) {
+        if ((in->x_new[s] == nullptr) != (in->g_new[s] == nullptr)) return CSA2_ERR_INVALID_ARG;
+        if (in->x_new[s] && !a16(in->x_new[s])) return CSA2_ERR_ALIGN;
+    }
+    const size_t need = csa2_layer_step_workspace(m);
+    if (!ws || ws_bytes < need) return CSA2_ERR_WORKSPACE;
+    if (!a16(ws)) return CSA2_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (ev) cudaEventRecord(ev[0], st);
+
+    // (1) every layer's window takes its token
+    WinAppend wa;
+    std::memset(&wa, 0, sizeof(wa));
+    wa.n = L;
+    wa.batch = B;
+    for (int l = 0; l < L; ++l) {
+        wa.tokens[l] = m->windows[l].tokens;
+        wa.count[l] = m->windows[l].count;
+        wa.tok[l] = in->win_tok[l];
+    }
+    rc = cuda_status(launch_window_append(wa, st));
+    if (rc) return rc;
+    if (ev) cudaEventRecord(ev[1], st);
+
+    // (2) the Full layer of each source writes its new token into the cache
+    for (int s = 0; s < m->n_sources; ++s) {
+        if (!in->x_new[s]) continue;
+        rc = cuda_status(launch_pack(view_of(m->caches[s]), in->x_new[s], false, in->g_new[s],
+                                     m->w_idx[s], 1, st));
+        if (rc) return rc;
+    }
+    if (ev) cudaEventRecord(ev[2], st);
+
+    // (3) every Full / Reindex layer scans its source with its own query
+    uint8_t* wsp = static_cast<uint8_t*>(ws);
+    const int cap = max_entries(m);
+    ScanBatch sb;
+    std::memset(&sb, 0, sizeof(sb));
+    sb.H_idx = m->H_idx;
+    sb.K = m->K;
+    for (int l = 0; l < L; ++l) {
+        const int md = m->mode[l];
+        if (md != CSA2_MODE_FULL && md != CSA2_MODE_REINDEX) continue;
+        ScanProblem& P = sb.p[sb.n++];
+        P.cache = view_of(m->caches[m->src[l]]);
+        P.q_idx = in->q_idx[l];
+        P.w = in->w[l];
+        P.idx_out = out->idx[l];
+        P.score_out = nullptr;
+        carve_scan(P, wsp, B, cap, m->H_idx);
+        wsp += topk_ws_one(B, cap, m->H_idx);
+    }
+    if (sb.n > 0) {
+        rc = cuda_status(launch_index_topk(sb, st, ev ? ev + 3 : nullptr));
+        if (rc) return rc;
+    } else if (ev) {
+        for (int i = 3; i < 6; ++i) cudaEventRecord(ev[i], st);
+    }
+
+    // (4) every layer attends; Reuse layers read the indices of idx_src
+    AttnBatch ab;
+    std::memset(&ab, 0, sizeof(ab));
+    ab.n = L;
+    ab.batch = B;
+    ab.H = m->H;
+    ab.Kmax = m->K;
+    ab.scale = m->scale;
+    const size_t units = attn_workspace_bytes(L, B, m->H, m->K) / ((D + 2) * sizeof(float));
+    ab.part_o = reinterpret_cast<float*>(wsp);
+    ab.part_ml = ab.part_o + units * D;
+    for (int l = 0; l < L; ++l) {
+        AttnProblem& P = ab.p[l];
+        const int md = m->mode[l];
+        P.q = in->q[l];
+        P.win = m->windows[l].tokens;
+        P.win_count = m->windows[l].count;
+        P.out = out->out[l];
+        if (md == CSA2_MODE_SWA_ONLY) {
+            P.K = 0;
+            P.idx = nullptr;
+        } else {
+            P.K = m->K;
+            P.cache = view_of(m->caches[m->src[l]]);
+            P.idx = out->idx[m->idx_src[l]];
+        }
+    }
+    return cuda_status(launch_sparse_attn(ab, st, ev ? ev + 6 : nullptr));
+}
+
+}  // namespace
+
+int csa2_layer_step(const csa2_model* m, const csa2_step_in* in, const csa2_step_out* out, void* ws,
+                    size_t ws_bytes, csa2_stream stream) {
+    return layer_step_impl(m, in, out, ws, ws_bytes, stream, nullptr);
+}
+
+int csa2_layer_step_profiled(const csa2_model* m, const csa2_step_in* in, const csa2_step_out* out,
+                             void* ws, size_t ws_bytes, csa2_stream stream, void* const* events) {
+    if (!events) return CSA2_ERR_INVALID_ARG;
+    cudaEvent_t ev[CSA2_STEP_EVENTS];
+    for (int i = 0; i < CSA2_STEP_EVENTS; ++i) {
+        if (!events[i]) return CSA2_ERR_INVALID_ARG;
+        ev[i] = (cudaEvent_t)events[i];
+    }
+    return layer_step_impl(m, in, out, ws, ws_bytes, stream, ev);
+}
+
+}  // extern "C"

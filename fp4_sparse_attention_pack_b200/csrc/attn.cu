@@ -1,0 +1,209 @@
+// Sparse + window attention ("la requête (main Q) lit les entrées
+// sélectionnées et le KV SWA local de la couche"; main KV "décompressé avant
+// l'attention"), the SWA ring write, and the split combine.
+//
+// Items of (problem, sequence): positions [0, K) are the selected entries
+// (index -1 or beyond n_entries is masked), positions [K, K + 128) the window
+// slots (slot >= min(count, 128) is masked).  The latent item is both key and
+// value.  Work unit = (problem, sequence, split of kSplit item positions):
+// the CTA dequantises its items into shared memory (fp32, exact), then each
+// warp takes one head at a time: scores (lane = item), softmax statistics by
+// warp shuffles, output accumulation (lane = 16 channels).  Partials
+// (max, sum, unnormalised output) are merged by k_attn_combine.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace csa2 {
+
+namespace {
+
+constexpr int kSplit = 64;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kStride = D + 1;  // padded item row (conflict-free column reads)
+
+__host__ __device__ inline int n_splits(int K) { return (K + WIN + kSplit - 1) / kSplit; }
+
+__global__ void __launch_bounds__(kThreads) k_attn_split(AttnBatch ab) {
+    extern __shared__ float sm[];
+    float* items = sm;                          // [kSplit][kStride]
+    float* qsh = items + kSplit * kStride;      // [kWarps][512]
+    __shared__ int valid[kSplit];
+    const AttnProblem& P = ab.p[blockIdx.z];
+    const int b = blockIdx.y;
+    const int split = blockIdx.x;
+    const int K = P.K;
+    const int ns = n_splits(K);
+    if (split >= ns) return;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int pos0 = split * kSplit;
+    const int wcount = P.win_count[b];
+    const int wlen = wcount < WIN ? (wcount < 0 ? 0 : wcount) : WIN;
+    const int n = (K > 0) ? entries_of(P.cache, b) : 0;
+
+    // ---- load + dequantise items (warp per item, lane = 16 channels = one scale)
+    for (int it = wid; it < kSplit; it += kWarps) {
+        const int pos = pos0 + it;
+        float* row = items + it * kStride;
+        int ok = 0;
+        if (pos < K) {
+            const int e = P.idx[(int64_t)b * K + pos];
+            if (e >= 0 && e < n) {
+                const int p = page_of(P.cache, b, e);
+                if (p >= 0) {
+                    ok = 1;
+                    const int64_t ent = (int64_t)p * PAGE + (e % PAGE);
+                    const uint2 cw = *reinterpret_cast<const uint2*>(P.cache.main_codes + ent * MCB + 8 * lane);
+                    const float s = e4m3_decode_pos(P.cache.main_scales[ent * MSB + lane]);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t by = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 0xFFu;
+                        row[16 * lane + 2 * k] = __fmul_rn(e2m1_decode(by & 15u), s);
+                        row[16 * lane + 2 * k + 1] = __fmul_rn(e2m1_decode(by >> 4), s);
+                    }
+                }
+            }
+        } else if (pos - K < wlen) {
+            ok = 1;
+            const uint16_t* src = P.win + ((int64_t)b * WIN + (pos - K)) * D + 16 * lane;
+            const uint4 u0 = *reinterpret_cast<const uint4*>(src);
+            const uint4 u1 = *reinterpret_cast<const uint4*>(src + 8);
+            const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                row[16 * lane + 2 * k] = __uint_as_float(w[k] << 16);
+                row[16 * lane + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+            }
+        }
+        if (lane == 0) valid[it] = ok;
+    }
+    __syncthreads();
+
+    // (problem, seq, split); the split stride is that of the largest K of the batch
+    const int64_t part = ((int64_t)blockIdx.z * ab.batch + b) * n_splits(ab.Kmax) + split;
+    float* q = qsh + wid * D;
+    for (int h = wid; h < ab.H; h += kWarps) {
+        const uint16_t* qs = P.q + ((int64_t)b * ab.H + h) * D;
+        for (int c = lane; c < D; c += 32) q[c] = bf16_bits_to_f32(qs[c]);
+        __syncwarp();
+        float s0 = 0.0f, s1 = 0.0f;
+        const float* r0 = items + lane * kStride;
+        const float* r1 = items + (lane + 32) * kStride;
+#pragma unroll 8
+        for (int c = 0; c < D; ++c) {
+            const float qc = q[c];
+            s0 = fmaf(qc, r0[c], s0);
+            s1 = fmaf(qc, r1[c], s1);
+        }
+        s0 = valid[lane] ? s0 * ab.scale : -INFINITY;
+        s1 = valid[lane + 32] ? s1 * ab.scale : -INFINITY;
+        float m = fmaxf(s0, s1);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float p0 = 0.0f, p1 = 0.0f;
+        if (m != -INFINITY) {
+            p0 = valid[lane] ? expf(s0 - m) : 0.0f;
+            p1 = valid[lane + 32] ? expf(s1 - m) : 0.0f;
+        }
+        float l = p0 + p1;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+        for (int j = 0; j < 32; ++j) {
+            const float pj0 = __shfl_sync(0xffffffffu, p0, j);
+            const float pj1 = __shfl_sync(0xffffffffu, p1, j);
+            const float* a0 = items + j * kStride + lane;
+            const float* a1 = items + (j + 32) * kStride + lane;
+            if (pj0 != 0.0f) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = fmaf(pj0, a0[32 * i], acc[i]);
+            }
+            if (pj1 != 0.0f) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = fmaf(pj1, a1[32 * i], acc[i]);
+            }
+        }
+        float* po = ab.part_o + (part * ab.H + h) * D;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) po[lane + 32 * i] = acc[i];
+        if (lane == 0) {
+            ab.part_ml[(part * ab.H + h) * 2 + 0] = m;
+            ab.part_ml[(part * ab.H + h) * 2 + 1] = l;
+        }
+        __syncwarp();
+    }
+}
+
+// out[b][h] = sum_s O_s e^(m_s - M) / sum_s l_s e^(m_s - M)
+__global__ void k_attn_combine(AttnBatch ab) {
+    const AttnProblem& P = ab.p[blockIdx.z];
+    const int b = blockIdx.y, h = blockIdx.x;
+    const int ns = n_splits(P.K);
+    const int64_t base = ((int64_t)blockIdx.z * ab.batch + b) * n_splits(ab.Kmax);
+    float M = -INFINITY;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, ab.part_ml[((base + s) * ab.H + h) * 2]);
+    float L = 0.0f;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M != -INFINITY) {
+        for (int s = 0; s < ns; ++s) {
+            const float m = ab.part_ml[((base + s) * ab.H + h) * 2];
+            if (m == -INFINITY) continue;
+            const float f = expf(m - M);
+            L += ab.part_ml[((base + s) * ab.H + h) * 2 + 1] * f;
+            const float* po = ab.part_o + ((base + s) * ab.H + h) * D;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] = fmaf(f, po[threadIdx.x + 128 * i], acc[i]);
+        }
+    }
+    float* o = P.out + ((int64_t)b * ab.H + h) * D;
+    const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[threadIdx.x + 128 * i] = acc[i] * inv;
+}
+
+__global__ void k_window_append(WinAppend wa) {
+    const int l = blockIdx.y, b = blockIdx.x;
+    const int cnt = wa.count[l][b];
+    __syncthreads();
+    const int slot = ((cnt % WIN) + WIN) % WIN;
+    const uint4* src = reinterpret_cast<const uint4*>(wa.tok[l] + (int64_t)b * D);
+    uint4* dst = reinterpret_cast<uint4*>(wa.tokens[l] + ((int64_t)b * WIN + slot) * D);
+    for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = src[i];
+    if (threadIdx.x == 0) wa.count[l][b] = cnt + 1;
+}
+
+}  // namespace
+
+size_t attn_workspace_bytes(int n_problems, int batch, int H, int Kmax) {
+    const size_t units = (size_t)n_problems * batch * n_splits(Kmax) * H;
+    return units * D * sizeof(float) + units * 2 * sizeof(float);
+}
+
+cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev) {
+    const size_t smem = sizeof(float) * (kSplit * kStride + kWarps * D);
+    static const bool attr_set = [smem] {
+        cudaFuncSetAttribute(k_attn_split, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        return true;
+    }();
+    (void)attr_set;
+    dim3 grid(n_splits(ab.Kmax), ab.batch, ab.n);
+    k_attn_split<<<grid, kThreads, smem, st>>>(ab);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (ev) cudaEventRecord(ev[0], st);
+    dim3 g2(ab.H, ab.batch, ab.n);
+    k_attn_combine<<<g2, 128, 0, st>>>(ab);
+    e = cudaGetLastError();
+    if (e == cudaSuccess && ev) cudaEventRecord(ev[1], st);
+    return e;
+}
+
+cudaError_t launch_window_append(const WinAppend& wa, cudaStream_t st) {
+    dim3 grid(wa.batch, wa.n);
+    k_window_append<<<grid, 64, 0, st>>>(wa);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,74 @@
+// Internal launchers of the CSA2 kernels (host side of csrc/*.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace csa2 {
+
+// ---- cache write
+cudaError_t launch_pack(const CacheView& c, const void* x, bool x_f32, const float* gates,
+                        const float* W, int T, cudaStream_t st);
+
+// ---- indexer
+// One scan problem: one indexer query set over one cache, for all sequences.
+struct ScanProblem {
+    CacheView cache;
+    const uint16_t* q_idx;  // bf16 [batch][H_idx][128]
+    const float* w;         // fp32 [batch][H_idx]
+    uint8_t* qc;            // workspace: MXFP4 query codes [batch][H_idx][64]
+    uint8_t* qs;            // workspace: E8M0 query scales [batch][H_idx][4]
+    float* scores;          // workspace: fp32 [batch][score_stride]
+    int64_t score_stride;
+    int32_t* idx_out;       // [batch][K]
+    float* score_out;       // nullable [batch][K]
+};
+
+constexpr int kMaxProblems = 64;
+struct ScanBatch {
+    ScanProblem p[kMaxProblems];
+    int n;
+    int H_idx;
+    int K;
+};
+
+// ev (nullable): events recorded after query quantisation, after the scan and
+// after Top-K (three cudaEvent_t).
+cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t* ev = nullptr);
+
+// ---- attention
+struct AttnProblem {
+    CacheView cache;          // valid when K > 0
+    const uint16_t* q;        // bf16 [batch][H][512]
+    const int32_t* idx;       // [batch][K] or null (K == 0)
+    const uint16_t* win;      // bf16 [batch][128][512]
+    const int32_t* win_count; // [batch]
+    float* out;               // fp32 [batch][H][512]
+    int K;                    // 0 for window-only layers
+};
+
+struct AttnBatch {
+    AttnProblem p[kMaxProblems];
+    int n;
+    int batch;
+    int H;
+    int Kmax;
+    float scale;
+    float* part_o;   // workspace partial outputs
+    float* part_ml;  // workspace partial (max, sum)
+};
+
+size_t attn_workspace_bytes(int n_problems, int batch, int H, int Kmax);
+// ev (nullable): events recorded after the split kernel and after the combine.
+cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev = nullptr);
+
+// ---- window
+struct WinAppend {
+    uint16_t* tokens[kMaxProblems];
+    int32_t* count[kMaxProblems];
+    const uint16_t* tok[kMaxProblems];
+    int n;
+    int batch;
+};
+cudaError_t launch_window_append(const WinAppend& wa, cudaStream_t st);
+
+}  // namespace csa2

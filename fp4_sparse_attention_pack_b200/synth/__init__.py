@@ -67,6 +67,8 @@ def _lib():
         _host.synth_normal_bf16.argtypes = [u64, u64, i64, vp, i64, vp]
         _host.synth_normal_scaled_f32.argtypes = [u64, u64, i64, ctypes.c_float, vp]
         _host.synth_uniform_f32.argtypes = [u64, u64, i64, vp]
+        _host.synth_normal_bf16_rows.argtypes = [u64, u64, u64, i64, i64, vp, i64, vp]
+        _host.synth_normal_f32_rows.argtypes = [u64, u64, u64, i64, i64, vp]
         _host.synth_u64_array.argtypes = [u64, u64, i64, vp]
     return _host
 
@@ -79,6 +81,8 @@ def _devlib():
         _dev.synth_dev_normal_bf16.argtypes = [u64, u64, i64, vp, i64, vp, vp]
         _dev.synth_dev_normal_scaled_f32.argtypes = [u64, u64, i64, ctypes.c_float, vp, vp]
         _dev.synth_dev_uniform_f32.argtypes = [u64, u64, i64, vp, vp]
+        _dev.synth_dev_normal_bf16_rows.argtypes = [u64, u64, u64, i64, i64, vp, i64, vp, vp]
+        _dev.synth_dev_normal_f32_rows.argtypes = [u64, u64, u64, i64, i64, vp, vp]
     return _dev
 
 
@@ -115,6 +119,25 @@ def normal_bf16(k: int, start: int, n: int, scale: np.ndarray | None = None) -> 
     return out
 
 
+def normal_bf16_rows(k: int, start: int, row_stride: int, rows: int, row_len: int,
+                     scale: np.ndarray | None = None) -> np.ndarray:
+    """bf16 bits [rows][row_len]: element start + r * row_stride + j."""
+    out = np.empty((rows, row_len), np.uint16)
+    if scale is not None:
+        scale = np.ascontiguousarray(scale, np.float32)
+        _lib().synth_normal_bf16_rows(k, start, row_stride, rows, row_len, scale.ctypes.data,
+                                      scale.size, out.ctypes.data)
+    else:
+        _lib().synth_normal_bf16_rows(k, start, row_stride, rows, row_len, None, 1, out.ctypes.data)
+    return out
+
+
+def normal_f32_rows(k: int, start: int, row_stride: int, rows: int, row_len: int) -> np.ndarray:
+    out = np.empty((rows, row_len), np.float32)
+    _lib().synth_normal_f32_rows(k, start, row_stride, rows, row_len, out.ctypes.data)
+    return out
+
+
 def uniform_f32(k: int, start: int, n: int) -> np.ndarray:
     out = np.empty(n, np.float32)
     _lib().synth_uniform_f32(k, start, n, out.ctypes.data)
@@ -139,6 +162,24 @@ def dev_normal_bf16(out, k: int, start: int, scale=None):
     nchan = scale.numel() if scale is not None else 1
     _check(_devlib().synth_dev_normal_bf16(k, start, n, sp, nchan, out.data_ptr(),
                                            torch.cuda.current_stream().cuda_stream))
+
+
+def dev_normal_bf16_rows(out, k: int, start: int, row_stride: int, rows: int, row_len: int,
+                         scale=None):
+    import torch
+    assert out.numel() == rows * row_len
+    sp = scale.data_ptr() if scale is not None else None
+    nchan = scale.numel() if scale is not None else 1
+    _check(_devlib().synth_dev_normal_bf16_rows(k, start, row_stride, rows, row_len, sp, nchan,
+                                                out.data_ptr(),
+                                                torch.cuda.current_stream().cuda_stream))
+
+
+def dev_normal_f32_rows(out, k: int, start: int, row_stride: int, rows: int, row_len: int):
+    import torch
+    assert out.numel() == rows * row_len
+    _check(_devlib().synth_dev_normal_f32_rows(k, start, row_stride, rows, row_len, out.data_ptr(),
+                                               torch.cuda.current_stream().cuda_stream))
 
 
 def dev_normal_scaled_f32(out, k: int, start: int, scale: float):

@@ -60,6 +60,29 @@ __global__ void k_uniform_f32(uint64_t key, uint64_t start, int64_t n, float* ou
         out[j] = __fmul_rn((float)(mix64(key + (start + j + 1) * kG) >> 40), 1.0f / 16777216.0f);
 }
 
+__global__ void k_normal_bf16_rows(uint64_t key, uint64_t start, uint64_t row_stride, int64_t rows,
+                                  int64_t row_len, const float* scale, int64_t nchan, uint16_t* out) {
+    const int64_t n = rows * row_len;
+    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < n;
+         j += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = j / row_len, c = j - r * row_len;
+        const uint64_t i = start + (uint64_t)r * row_stride + (uint64_t)c;
+        float v = normal_f32(key, i);
+        if (scale) v = __fmul_rn(v, scale[i % (uint64_t)nchan]);
+        out[j] = f32_to_bf16_rne(v);
+    }
+}
+
+__global__ void k_normal_f32_rows(uint64_t key, uint64_t start, uint64_t row_stride, int64_t rows,
+                                  int64_t row_len, float* out) {
+    const int64_t n = rows * row_len;
+    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < n;
+         j += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = j / row_len, c = j - r * row_len;
+        out[j] = normal_f32(key, start + (uint64_t)r * row_stride + (uint64_t)c);
+    }
+}
+
 int grid_for(int64_t n) {
     int64_t g = (n + 255) / 256;
     if (g > 148 * 32) g = 148 * 32;
@@ -79,6 +102,24 @@ extern "C" int synth_dev_normal_scaled_f32(uint64_t key, uint64_t start, int64_t
                                            float* out, cudaStream_t stream) {
     if (n <= 0) return 0;
     k_normal_scaled_f32<<<grid_for(n), 256, 0, stream>>>(key, start, n, scale, out);
+    return (int)cudaGetLastError();
+}
+
+extern "C" int synth_dev_normal_bf16_rows(uint64_t key, uint64_t start, uint64_t row_stride,
+                                          int64_t rows, int64_t row_len, const float* scale,
+                                          int64_t nchan, uint16_t* out, cudaStream_t stream) {
+    if (rows * row_len <= 0) return 0;
+    k_normal_bf16_rows<<<grid_for(rows * row_len), 256, 0, stream>>>(key, start, row_stride, rows,
+                                                                     row_len, scale, nchan, out);
+    return (int)cudaGetLastError();
+}
+
+extern "C" int synth_dev_normal_f32_rows(uint64_t key, uint64_t start, uint64_t row_stride,
+                                         int64_t rows, int64_t row_len, float* out,
+                                         cudaStream_t stream) {
+    if (rows * row_len <= 0) return 0;
+    k_normal_f32_rows<<<grid_for(rows * row_len), 256, 0, stream>>>(key, start, row_stride, rows,
+                                                                    row_len, out);
     return (int)cudaGetLastError();
 }
 

@@ -87,6 +87,27 @@ void synth_normal_scaled_f32(uint64_t key, uint64_t start, int64_t n, float scal
     for (int64_t j = 0; j < n; ++j) out[j] = normal_f32(key, start + (uint64_t)j) * scale;
 }
 
+/* 2-D form: out[r][j] = element start + r * row_stride + j, j < row_len. */
+void synth_normal_bf16_rows(uint64_t key, uint64_t start, uint64_t row_stride, int64_t rows,
+                            int64_t row_len, const float* scale, int64_t nchan, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < row_len; ++j) {
+            uint64_t i = start + (uint64_t)r * row_stride + (uint64_t)j;
+            float v = normal_f32(key, i);
+            if (scale) v = v * scale[i % (uint64_t)nchan];
+            out[r * row_len + j] = f32_to_bf16_rne(v);
+        }
+}
+
+void synth_normal_f32_rows(uint64_t key, uint64_t start, uint64_t row_stride, int64_t rows,
+                           int64_t row_len, float* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < row_len; ++j)
+            out[r * row_len + j] = normal_f32(key, start + (uint64_t)r * row_stride + (uint64_t)j);
+}
+
 void synth_uniform_f32(uint64_t key, uint64_t start, int64_t n, float* out) {
 #pragma omp parallel for schedule(static)
     for (int64_t j = 0; j < n; ++j)

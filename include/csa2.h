@@ -1,0 +1,289 @@
+/*
+ * csa2.h -- C ABI of the CSA2 sparse-decode library for NVIDIA B200 (sm_100a).
+ *
+ * CSA2 ("DeepSeek-V4.1-Flash, expliqué pas à pas", CSA2 chapter; "Résumé
+ * exécutif", section "CSA2 -- le partage du cache entre couches") gives each
+ * layer a global branch over a compressed, shared cache and a local 128-token
+ * sliding-window (SWA) branch.  This library implements the decode hot path:
+ *
+ *   csa2_pack_cache   cache write: disjoint token groups of m = 2 (or m = 1)
+ *                     compressed into one entry, stored as E2M1 with one E4M3
+ *                     scale per 16 channels (288 B), plus an indexer key
+ *                     projected from that entry and stored as OCP MXFP4
+ *                     (E2M1 + one E8M0 scale per 32 channels, 68 B);
+ *   csa2_index_topk   indexer scan: score every entry from an MXFP4 indexer
+ *                     query, keep the K best per sequence;
+ *   csa2_sparse_attn  attention of the main query over the K selected entries
+ *                     (dequantised) joined with the layer's own window;
+ *   csa2_window_append  SWA ring write of the current token;
+ *   csa2_layer_step   one decode step of a whole stack of layers under the
+ *                     static Full / Reindex / Reuse mode table.
+ *
+ * Conventions (all entry points):
+ *   - Every tensor is caller-owned DEVICE memory unless stated otherwise; the
+ *     library allocates nothing and keeps no pointer after a call returns.
+ *     Scratch memory is a caller-provided workspace whose size the matching
+ *     *_workspace function reports (0 is a valid answer).
+ *   - Calls are asynchronous on the caller's CUDA stream (NULL = the legacy
+ *     default stream) and never synchronise the device, so they may be
+ *     captured in a CUDA graph.  Host-side descriptor structs are read during
+ *     the call only.
+ *   - Return value: CSA2_OK (0) or a negative csa2_status.  Arguments are
+ *     validated before anything is launched: on an error return nothing has
+ *     been enqueued.  No call aborts, throws or traps.
+ *   - Conditions only the device can see (a full cache, a page id outside the
+ *     pool) never fault: the kernel skips the write and ORs a CSA2_DEVERR_*
+ *     bit into the cache's sticky status word, which the caller reads back.
+ *   - Device pointers must be 16-byte aligned (CSA2_ERR_ALIGN otherwise).
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Fixed dimensions: latent D = 512, indexer dim 128, window 128,
+ *     page = 64 entries.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* csa2_stream; /* same type as cudaStream_t */
+
+enum {
+    CSA2_D = 512,                 /* main latent channels */
+    CSA2_D_IDX = 128,             /* indexer query / key dim */
+    CSA2_WIN = 128,               /* sliding window (n_win) */
+    CSA2_PAGE = 64,               /* entries per cache page */
+    CSA2_MAIN_CODE_BYTES = 256,   /* 512 E2M1 codes */
+    CSA2_MAIN_SCALE_BYTES = 32,   /* 32 E4M3 scales (one per 16 channels) */
+    CSA2_IDX_CODE_BYTES = 64,     /* 128 E2M1 codes */
+    CSA2_IDX_SCALE_BYTES = 4,     /* 4 E8M0 scales (one per 32 channels) */
+    CSA2_MAX_K = 2048,
+    CSA2_MAX_H = 128,
+    CSA2_MAX_H_IDX = 64,
+    CSA2_MAX_LAYERS = 64,
+    CSA2_MAX_SOURCES = 8
+};
+
+typedef enum {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = -1, /* null pointer, size out of range, bad mode table */
+    CSA2_ERR_ALIGN = -2,       /* a device pointer is not 16-byte aligned */
+    CSA2_ERR_UNSUPPORTED = -3, /* a size this build does not handle */
+    CSA2_ERR_CUDA = -4,        /* a CUDA launch or runtime call failed */
+    CSA2_ERR_TIMEOUT = -5,     /* a bounded device wait gave up (reported via status) */
+    CSA2_ERR_WORKSPACE = -6    /* ws is NULL or smaller than the *_workspace size */
+} csa2_status;
+
+typedef enum {
+    CSA2_MODE_SWA_ONLY = 0, /* window only (layers 0 and 1 of the model) */
+    CSA2_MODE_FULL = 1,     /* computes main cache, indexer keys and Top-K */
+    CSA2_MODE_REINDEX = 2,  /* reuses cache and keys, recomputes Top-K */
+    CSA2_MODE_REUSE = 3     /* reuses cache, keys and Top-K indices */
+} csa2_mode;
+
+typedef enum { CSA2_DTYPE_BF16 = 0, CSA2_DTYPE_F32 = 1 } csa2_dtype;
+
+/* Sticky device error bits (csa2_cache.status). */
+#define CSA2_DEVERR_CAPACITY 0x1u /* an append would exceed max_pages * 64 entries */
+#define CSA2_DEVERR_PAGE 0x2u     /* a page-table entry is outside [0, num_pages) */
+#define CSA2_DEVERR_COUNT 0x4u    /* n_entries outside [0, max_pages * 64] */
+#define CSA2_DEVERR_TIMEOUT 0x8u  /* a bounded device wait gave up */
+
+/*
+ * One source layer's compressed cache for `batch` sequences, paged.
+ * ("Le cache KV en FP4": main entry = 512 E2M1 values + one E4M3 scale per 16
+ * channels = 256 + 32 B; indexer key = 128 E2M1 + one E8M0 per 32 = 64 + 4 B.)
+ *
+ * Logical entry e of sequence b lives in physical page
+ * p = page_table[b * max_pages + e / 64], slot e % 64, and its bytes are
+ *   main_codes [p][slot][256]  channel 2i in the low nibble of byte i,
+ *                              channel 2i+1 in the high nibble;
+ *   main_scales[p][slot][32]   E4M3, byte j scales channels 16j..16j+15;
+ *   idx_codes  [p][slot][64]   same nibble order over the 128 key channels;
+ *   idx_scales [p][slot][4]    E8M0, byte j scales channels 32j..32j+31.
+ * Each pool is num_pages * 64 * (bytes per entry) long.
+ *
+ * Ratio-2 sources keep one pending token per sequence (pend_x fp32[512],
+ * pend_g, pend_valid) until its pair arrives.  `status` is a device uint32
+ * the kernels OR CSA2_DEVERR_* bits into; the caller clears it.
+ */
+typedef struct {
+    uint8_t* main_codes;
+    uint8_t* main_scales;
+    uint8_t* idx_codes;
+    uint8_t* idx_scales;
+    const int32_t* page_table; /* [batch][max_pages] */
+    int32_t* n_entries;        /* [batch] entries stored */
+    float* pend_x;             /* [batch][512] */
+    float* pend_g;             /* [batch] */
+    int32_t* pend_valid;       /* [batch] 0 or 1 */
+    uint32_t* status;          /* [1] */
+    int32_t batch;
+    int32_t max_pages;         /* pages per sequence (page-table row length) */
+    int32_t num_pages;         /* pages in each pool */
+    int32_t ratio;             /* tokens per entry: 2 (encoder) or 1 (decoder) */
+} csa2_cache;
+
+/*
+ * One layer's SWA window for `batch` sequences ("une branche locale SWA qui
+ * maintient le KV SWA des 128 derniers tokens"): a ring of 128 bf16 tokens of
+ * 512 channels.  Token number t (0-based, counted per sequence) sits in slot
+ * t % 128; count[b] tokens were appended, the first min(count[b], 128) slots
+ * are valid.  Attention is order-free, so the ring needs no rotation.
+ */
+typedef struct {
+    uint16_t* tokens; /* bf16 [batch][128][512] */
+    int32_t* count;   /* [batch] */
+    int32_t batch;
+} csa2_window;
+
+/* Library version, (major << 16) | minor. */
+int csa2_version(void);
+
+/* Static string for a csa2_status value (never NULL). */
+const char* csa2_strerror(int status);
+
+/*
+ * Cache write ("CSA2 supprime le chevauchement" -- disjoint groups; "CSA2
+ * obtient l'indexer K par une simple projection du main KV"; "Le cache KV en
+ * FP4").  Appends T_new tokens to every sequence of `cache`:
+ *   x       [batch][T_new][512] tokens, bf16 or fp32 per x_dtype (the
+ *           post-RoPE latent of the source layer);
+ *   gates   fp32 [batch][T_new], one gate logit per token;
+ *   w_idx   fp32 [512][128] row-major indexer projection of this source.
+ * Ratio 2: tokens pair up in arrival order with the pending token first; each
+ * pair (x0, x1) becomes e = w0*x0 + w1*x1, (w0, w1) = softmax(g0, g1), in fp32
+ * with the library's fixed exp (Cody-Waite reduction + degree-7 Taylor).  Ratio
+ * 1: each token is an entry.  Each entry is packed (per 16 channels:
+ * s = E4M3(amax/6) nearest-even, codes = E2M1(e/s) nearest-even saturating),
+ * its indexer key is k_o = sum_c w_idx[c][o] * deq_c accumulated in fp32 fma
+ * order c = 0..511, and k is packed to MXFP4 (per 32: X = floor(log2 amax)-2,
+ * codes = E2M1(k * 2^-X)).  Updates n_entries and the pending slot.
+ * Errors: INVALID_ARG (null, T_new < 0, bad dtype/ratio), ALIGN, CUDA.  A full
+ * cache sets CSA2_DEVERR_CAPACITY and leaves that sequence unchanged.
+ */
+int csa2_pack_cache(const csa2_cache* cache, const void* x, int x_dtype, const float* gates,
+                    const float* w_idx, int T_new, csa2_stream stream);
+
+/* Workspace bytes csa2_index_topk needs for these sizes. */
+size_t csa2_index_topk_workspace(int batch, int max_entries, int H_idx, int K);
+
+/*
+ * Indexer scan + Top-K ("un indexeur léger : il note chaque entrée du main KV
+ * en combinant une indexer Q et une indexer K, puis garde les 512 meilleures";
+ * indexer queries and keys in OCP MXFP4).  For every sequence b:
+ *   score[e] = sum_h w[b][h] * max(0, qhat[b][h] . khat[e]),  e < n_entries[b],
+ * qhat = MXFP4 of q_idx (same rule as the keys), khat the stored keys.
+ * The K highest scores are kept (equal scores: lower index first); idx_out
+ * [batch][K] receives them in increasing index order followed by -1 padding
+ * when n_entries < K.  score_out (nullable) [batch][K] receives the matching
+ * fp32 scores (0 for padding).
+ *   q_idx  bf16 [batch][H_idx][128];  w fp32 [batch][H_idx].
+ * H_idx in 1..64, K in 1..2048.  ws must hold
+ * csa2_index_topk_workspace(batch, max_pages*64, H_idx, K) bytes.
+ */
+int csa2_index_topk(const csa2_cache* cache, const uint16_t* q_idx, const float* w, int H_idx,
+                    int K, int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
+                    csa2_stream stream);
+
+/* Workspace bytes csa2_sparse_attn needs for these sizes. */
+size_t csa2_sparse_attn_workspace(int batch, int H, int K);
+
+/*
+ * Sparse + window attention ("l'attention principale : la requête (main Q)
+ * lit les entrées sélectionnées et le KV SWA local de la couche"; entries are
+ * "décompressées avant l'attention").  For every sequence b and head h:
+ *   items = dequantised entries idx[b][0..K) (index -1 skipped; indices at or
+ *           beyond n_entries[b] skipped) followed by the valid window tokens;
+ *   out[b][h] = sum_j softmax_j(scale * q[b][h] . item_j) * item_j
+ * (the latent serves as key and value).  No items gives zeros.
+ *   q     bf16 [batch][H][512];  idx int32 [batch][K] (may be NULL when K = 0);
+ *   out   fp32 [batch][H][512].
+ * H in 1..128, K in 0..2048.  `cache` may be NULL when K = 0.
+ */
+int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const int32_t* idx, int K,
+                     const csa2_window* win, float scale, float* out, void* ws, size_t ws_bytes,
+                     csa2_stream stream);
+
+/* SWA ring write: tok bf16 [batch][512] goes to slot count % 128; count += 1. */
+int csa2_window_append(const csa2_window* win, const uint16_t* tok, csa2_stream stream);
+
+/*
+ * A stack of layers and its static mode table ("Chaque couche CSA2 reçoit, de
+ * façon statique, l'un des trois modes"; "Résumé exécutif" mode table):
+ *   mode[l]     csa2_mode of layer l;
+ *   src[l]      the source cache layer l reads (ignored for SWA_ONLY);
+ *   idx_src[l]  for REUSE: the earlier FULL/REINDEX layer of the same source
+ *               whose indices it reuses; for FULL/REINDEX: l itself.
+ * Every source is written by exactly one FULL layer.  Host arrays; the caches,
+ * w_idx pointers and windows they list are device memory as above.
+ */
+typedef struct {
+    int32_t n_layers;
+    int32_t n_sources;
+    const int32_t* mode;            /* host [n_layers] */
+    const int32_t* src;             /* host [n_layers] */
+    const int32_t* idx_src;         /* host [n_layers] */
+    const csa2_cache* caches;       /* host [n_sources] */
+    const float* const* w_idx;      /* host [n_sources] -> device fp32 [512][128] */
+    const csa2_window* windows;     /* host [n_layers] */
+    int32_t batch;
+    int32_t H;                      /* main query heads */
+    int32_t H_idx;                  /* indexer heads */
+    int32_t K;                      /* Top-K */
+    float scale;                    /* softmax scale (1/sqrt(512) in the tests) */
+} csa2_model;
+
+/* Per-step inputs: host arrays of device pointers. */
+typedef struct {
+    const uint16_t* const* x_new; /* [n_sources] -> bf16 [batch][512]: the new token */
+    const float* const* g_new;    /* [n_sources] -> fp32 [batch]: its gate logit */
+    const uint16_t* const* q;     /* [n_layers] -> bf16 [batch][H][512] */
+    const uint16_t* const* q_idx; /* [n_layers] -> bf16 [batch][H_idx][128] (FULL/REINDEX) */
+    const float* const* w;        /* [n_layers] -> fp32 [batch][H_idx] (FULL/REINDEX) */
+    const uint16_t* const* win_tok; /* [n_layers] -> bf16 [batch][512]: this token's SWA KV */
+} csa2_step_in;
+
+/* Per-step outputs: host arrays of device pointers. */
+typedef struct {
+    float* const* out;   /* [n_layers] -> fp32 [batch][H][512] */
+    int32_t* const* idx; /* [n_layers] -> int32 [batch][K] for FULL/REINDEX layers (others
+                            unused and may be NULL) */
+} csa2_step_out;
+
+/* Workspace bytes csa2_layer_step needs for this model. */
+size_t csa2_layer_step_workspace(const csa2_model* model);
+
+/*
+ * One decode step of every layer.  Order: (1) each layer's window takes its
+ * token; (2) each source takes its new token (an entry is written when a
+ * ratio-2 pair completes); (3) every FULL/REINDEX layer scans its source with
+ * its own indexer query and keeps the Top-K; (4) every layer attends: REUSE
+ * layers over the indices of idx_src, SWA_ONLY layers over the window only.
+ * Errors as the per-op calls; INVALID_ARG for an inconsistent mode table.
+ */
+int csa2_layer_step(const csa2_model* model, const csa2_step_in* in, const csa2_step_out* out,
+                    void* ws, size_t ws_bytes, csa2_stream stream);
+
+/*
+ * Measurement variant of csa2_layer_step: identical work, and in addition
+ * records CUDA events on `stream` at the phase boundaries.  `events` is a host
+ * array of CSA2_STEP_EVENTS cudaEvent_t handles (as void*) created by the caller
+ * with timing enabled:
+ *   [0] start            [1] after window append  [2] after cache write
+ *   [3] after query quantisation                  [4] after the indexer scan
+ *   [5] after Top-K      [6] after attention      [7] after the split combine
+ * A phase with nothing to do gives two events with no work between them.
+ */
+#define CSA2_STEP_EVENTS 8
+int csa2_layer_step_profiled(const csa2_model* model, const csa2_step_in* in,
+                             const csa2_step_out* out, void* ws, size_t ws_bytes,
+                             csa2_stream stream, void* const* events);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */

@@ -1,0 +1,43 @@
+"""Parity criteria of the CUDA path against the oracle (stated once, used by all GPU tests).
+
+* packed caches: bit-exact, byte for byte, in logical entry order;
+* Top-K: the GPU's index set equals the oracle's except for entries whose
+  oracle score lies within TOPK_REL of the oracle's K-th score (their count is
+  returned); indices distinct, within [0, n), increasing, padded with -1;
+* attention: per (sequence, head) row, max_c |o - r| / max_c |r| <= ATTN_REL,
+  the oracle evaluated on the GPU's own index set.
+"""
+import numpy as np
+
+TOPK_REL = 1e-5
+ATTN_REL = 2e-3
+
+
+def check_topk(gpu_idx: np.ndarray, ref_scores: np.ndarray, K: int) -> int:
+    """Assert the Top-K criterion for one sequence; return the tie-band count."""
+    n = ref_scores.size
+    gpu_idx = np.asarray(gpu_idx, np.int64)
+    m = min(K, n)
+    assert np.all(gpu_idx[m:] == -1), "padding must be -1"
+    g = gpu_idx[:m]
+    assert np.all((g >= 0) & (g < n)), "index out of range"
+    assert np.all(np.diff(g) > 0), "indices must be distinct and increasing"
+    if m == 0:
+        return 0
+    order = sorted(range(n), key=lambda i: (-ref_scores[i], i)) if n < 4096 else \
+        np.lexsort((np.arange(n), -ref_scores))
+    ref_set = set(int(i) for i in order[:m])
+    kth = ref_scores[order[m - 1]]
+    band = np.abs(ref_scores - kth) <= TOPK_REL * max(abs(kth), 1e-30)
+    diff = ref_set.symmetric_difference(set(int(i) for i in g))
+    bad = [i for i in diff if not band[i]]
+    assert not bad, f"{len(bad)} Top-K entries differ outside the tie band, e.g. {bad[:5]}"
+    return len(diff)
+
+
+def attn_rel_err(out: np.ndarray, ref: np.ndarray) -> float:
+    """max over rows of max_c |o - r| / max_c |r| (rows = all leading dims)."""
+    o = np.asarray(out, np.float64).reshape(-1, out.shape[-1])
+    r = np.asarray(ref, np.float64).reshape(-1, ref.shape[-1])
+    den = np.maximum(np.abs(r).max(axis=1), 1e-30)
+    return float((np.abs(o - r).max(axis=1) / den).max())

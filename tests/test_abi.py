@@ -1,0 +1,99 @@
+"""The C ABI library builds for sm_100a, loads without a GPU and exports every
+function include/csa2.h declares; host-side argument checks return errors
+before anything is launched (no GPU needed: nothing reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def capi():
+    from fp4_sparse_attention_pack_b200 import _build
+    _build.build()
+    import fp4_sparse_attention_pack_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "csa2.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa2_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ("csa2_pack_cache", "csa2_index_topk", "csa2_sparse_attn", "csa2_layer_step",
+              "csa2_window_append", "csa2_version", "csa2_strerror"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(capi):
+    lib = capi.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.csa2_version() >= 1
+    assert lib.csa2_strerror(-1) == b"invalid argument"
+
+
+def test_argument_checks_fail_before_launch(capi):
+    lib = capi.lib()
+    c = capi.csa2_cache()
+    # null cache pointers -> invalid argument, nothing enqueued
+    assert lib.csa2_pack_cache(ctypes.byref(c), None, 0, None, None, 4, None) == -1
+    c = capi.csa2_cache(*([16] * 10), 1, 1, 1, 2)
+    assert lib.csa2_pack_cache(ctypes.byref(c), ctypes.c_void_p(16), 7, ctypes.c_void_p(16),
+                               ctypes.c_void_p(16), 4, None) == -1          # bad dtype
+    c2 = capi.csa2_cache(*([16] * 9 + [17]), 1, 1, 1, 2)
+    assert lib.csa2_pack_cache(ctypes.byref(c2), ctypes.c_void_p(16), 0, ctypes.c_void_p(16),
+                               ctypes.c_void_p(16), 4, None) == -2          # misaligned
+    c3 = capi.csa2_cache(*([16] * 10), 1, 1, 1, 3)
+    assert lib.csa2_pack_cache(ctypes.byref(c3), ctypes.c_void_p(16), 0, ctypes.c_void_p(16),
+                               ctypes.c_void_p(16), 4, None) == -1          # bad ratio
+    # K and H_idx ranges; workspace too small
+    assert lib.csa2_index_topk(ctypes.byref(c), ctypes.c_void_p(16), ctypes.c_void_p(16), 65, 8,
+                               ctypes.c_void_p(16), None, None, 0, None) == -1
+    assert lib.csa2_index_topk(ctypes.byref(c), ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 4096,
+                               ctypes.c_void_p(16), None, None, 0, None) == -1
+    assert lib.csa2_index_topk(ctypes.byref(c), ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 8,
+                               ctypes.c_void_p(16), None, None, 0, None) == -6
+    w = capi.csa2_window(16, 16, 1)
+    assert lib.csa2_sparse_attn(None, ctypes.c_void_p(16), 4, None, 0, ctypes.byref(w), 0.1,
+                                ctypes.c_void_p(16), None, 0, None) == -6
+    assert lib.csa2_sparse_attn(None, ctypes.c_void_p(16), 0, None, 0, ctypes.byref(w), 0.1,
+                                ctypes.c_void_p(16), None, 0, None) == -1
+    assert capi.index_topk_workspace(2, 1024, 64, 512) > 2 * 1024 * 4
+    assert capi.sparse_attn_workspace(2, 64, 512) > 0
+
+
+def test_mode_table_validation(capi):
+    import numpy as np
+    from fp4_sparse_attention_pack_b200 import workloads as W
+    lib = capi.lib()
+
+    def model(mode, src, idx_src, ratios=(2,)):
+        L, S = len(mode), len(ratios)
+        caches = (capi.csa2_cache * S)(*[capi.csa2_cache(*([16] * 10), 1, 1, 1, r) for r in ratios])
+        wins = (capi.csa2_window * L)(*[capi.csa2_window(16, 16, 1) for _ in range(L)])
+        ws = (ctypes.c_void_p * S)(*([16] * S))
+        keep = [(ctypes.c_int32 * L)(*mode), (ctypes.c_int32 * L)(*src), (ctypes.c_int32 * L)(*idx_src)]
+        m = capi.csa2_model(L, S, keep[0], keep[1], keep[2], caches, ws, wins, 1, 4, 4, 8, 0.04)
+        return m, (caches, wins, ws, keep)
+
+    ok, keep = model([W.SWA_ONLY, W.FULL, W.REINDEX, W.REUSE], [0, 0, 0, 0], [0, 1, 2, 2])
+    assert capi.layer_step_workspace(ok) > 0
+    for mode, src, idx_src in [
+        ([W.REUSE, W.FULL], [0, 0], [1, 1]),            # reuse names a later layer
+        ([W.FULL, W.FULL], [0, 0], [0, 1]),             # two writers of one source
+        ([W.REINDEX, W.FULL], [0, 0], [0, 1]),          # reindex before the source exists
+        ([W.FULL, 7], [0, 0], [0, 1]),                  # unknown mode
+        ([W.SWA_ONLY], [0], [0]),                       # a source nobody writes
+    ]:
+        bad, keep2 = model(mode, src, idx_src)
+        assert capi.layer_step_workspace(bad) == 0
+        sin, sout = capi.csa2_step_in(), capi.csa2_step_out()
+        assert lib.csa2_layer_step(ctypes.byref(bad), ctypes.byref(sin), ctypes.byref(sout),
+                                   ctypes.c_void_p(256), 1 << 30, None) == -1
