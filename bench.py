@@ -39,7 +39,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--workload", default=None,
+                    help="a profiling case of workloads.PROFILE_WORKLOADS instead of --config")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=5)
     return ap.parse_args()
 
@@ -277,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
-    base = W.WORKLOADS[args.config]
+    base = W.PROFILE_WORKLOADS[args.workload] if args.workload else W.WORKLOADS[args.config]
     wl = W.small(base, seed=base.seed + 1000 * rank)  # each rank: its own batch of sequences
     extra = args.warmup + args.steps + 2 * args.profile_steps + 8
     dm = engine.DecodeModel(wl, dev, steps_capacity=extra)
@@ -339,6 +342,9 @@ def run_ours(args, rank, world, local_rank):
                                              ctypes.POINTER(csa.csa2_step_out), ctypes.c_void_p,
                                              ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]
     phase = [[] for _ in names]
+    for x in evs:  # torch creates the CUDA event on first record
+        x.record(stream)
+    torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for i in range(args.profile_steps):
             e = evs[8 * i:8 * i + 8]
@@ -364,7 +370,7 @@ def run_ours(args, rank, world, local_rank):
     host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
     h2d = sum(t.numel() * t.element_size() for t in ins)
     d2h = sum(t.numel() * t.element_size() for t in outs)
-    e2e_steps = max(3, min(args.steps, 30))
+    e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 30))
     torch.cuda.synchronize()
     barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -378,7 +384,7 @@ def run_ours(args, rank, world, local_rank):
                 h.copy_(d, non_blocking=True)
         f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps if e2e_steps else float("nan")
     if world > 1:
         tt = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -421,7 +427,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks.summary(t_wall0, t_wall1),
         "device_status": status,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not args.workload:
         line["cpu_baseline"] = cpu_baseline(W.WORKLOADS[args.config])
     print(json.dumps(line), flush=True)
 

@@ -134,6 +134,14 @@ WORKLOADS = {
 }
 
 
+# Profiling cases: one kernel at a size whose inputs exceed L2 (126 MB) while the
+# device holds a few GB at most.
+PROFILE_WORKLOADS = {
+    # one Full layer over 32 sequences x 65,536 entries: 142 MB of indexer keys per scan
+    "scan32": Workload("scan32_1layer_b32_128k", 5, 32, 131072, single_full(), 64, 64, 512, 4),
+}
+
+
 def small(wl: Workload, **kw) -> Workload:
     """A reduced copy of a workload (same recipe, smaller sizes)."""
     return dataclasses.replace(wl, **kw)

@@ -162,8 +162,10 @@ const char* csa2_strerror(int status);
  * its indexer key is k_o = sum_c w_idx[c][o] * deq_c accumulated in fp32 fma
  * order c = 0..511, and k is packed to MXFP4 (per 32: X = floor(log2 amax)-2,
  * codes = E2M1(k * 2^-X)).  Updates n_entries and the pending slot.
- * Errors: INVALID_ARG (null, T_new < 0, bad dtype/ratio), ALIGN, CUDA.  A full
- * cache sets CSA2_DEVERR_CAPACITY and leaves that sequence unchanged.
+ * Errors: INVALID_ARG (null, T_new < 0 or above twice the capacity
+ * max_pages * 64, bad dtype/ratio), ALIGN, CUDA.  An append that does not fit
+ * a sequence's remaining capacity sets CSA2_DEVERR_CAPACITY and leaves that
+ * sequence unchanged.
  */
 int csa2_pack_cache(const csa2_cache* cache, const void* x, int x_dtype, const float* gates,
                     const float* w_idx, int T_new, csa2_stream stream);

@@ -174,12 +174,20 @@ def test_pack_rounding_ties(csa):
 def test_pack_capacity_error_sets_status(csa):
     wl = W.WORKLOADS[0]
     dc = csa.engine.DeviceCache(1, 1, 2, DEV)  # 64 entries
-    x = W.tokens(wl, 0, 0, 0, 200)[None]
-    g = W.gates(wl, 0, 0, 0, 200)[None]
-    csa.pack_cache(dc.desc, bf16_dev(x), f32_dev(g), f32_dev(W.w_idx(wl, 0)))
+    Wd = f32_dev(W.w_idx(wl, 0))
+    x = W.tokens(wl, 0, 0, 0, 140)[None]
+    g = W.gates(wl, 0, 0, 0, 140)[None]
+    csa.pack_cache(dc.desc, bf16_dev(x[:, :100]), f32_dev(g[:, :100]), Wd)  # 50 entries
+    torch.cuda.synchronize()
+    assert dc.n_entries.item() == 50 and dc.status_bits() == 0
+    csa.pack_cache(dc.desc, bf16_dev(x[:, 100:]), f32_dev(g[:, 100:]), Wd)  # 20 more: full
     torch.cuda.synchronize()
     assert dc.status_bits() & csa.DEVERR_CAPACITY
-    assert dc.n_entries.item() == 0
+    assert dc.n_entries.item() == 50  # that sequence is left unchanged
+    # an append more than twice the capacity is refused on the host, nothing launched
+    with pytest.raises(csa.Csa2Error):
+        csa.pack_cache(dc.desc, bf16_dev(W.tokens(wl, 0, 0, 0, 200)[None]),
+                       f32_dev(W.gates(wl, 0, 0, 0, 200)[None]), Wd)
 
 
 # ---------------------------------------------------------------- indexer
