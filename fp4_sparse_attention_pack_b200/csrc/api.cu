@@ -43,18 +43,7 @@ int check_window(const csa2_window* w, int batch) {
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
 
 size_t topk_ws_one(int batch, int max_entries, int H_idx) {
-    return align_up((size_t)batch * H_idx * ICB) + align_up((size_t)batch * H_idx * ISB) +
-           align_up((size_t)batch * max_entries * sizeof(float));
-}
-
-// Carve one scan problem's scratch out of ws.
-void carve_scan(ScanProblem& P, uint8_t* ws, int batch, int max_entries, int H_idx) {
-    P.qc = ws;
-    ws += align_up((size_t)batch * H_idx * ICB);
-    P.qs = ws;
-    ws += align_up((size_t)batch * H_idx * ISB);
-    P.scores = reinterpret_cast<float*>(ws);
-    P.score_stride = max_entries;
+    return scan_workspace_bytes(1, batch, max_entries, H_idx);
 }
 
 }  // namespace
@@ -119,7 +108,7 @@ int csa2_index_topk(const csa2_cache* cache, const uint16_t* q_idx, const float*
     P.w = w;
     P.idx_out = idx_out;
     P.score_out = score_out;
-    carve_scan(P, static_cast<uint8_t*>(ws), cache->batch, cap, H_idx);
+    carve_scan_workspace(sb, static_cast<uint8_t*>(ws), cache->batch, cap);
     return cuda_status(launch_index_topk(sb, (cudaStream_t)stream));
 }
 
@@ -246,7 +235,7 @@ int n_scans(const csa2_model* m) {
 
 size_t csa2_layer_step_workspace(const csa2_model* m) {
     if (check_model(m)) return 0;
-    return (size_t)n_scans(m) * topk_ws_one(m->batch, max_entries(m), m->H_idx) +
+    return align_up(scan_workspace_bytes(n_scans(m), m->batch, max_entries(m), m->H_idx)) +
            align_up(attn_workspace_bytes(m->n_layers, m->batch, m->H, m->K));
 }
 
@@ -318,9 +307,9 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
         P.w = in->w[l];
         P.idx_out = out->idx[l];
         P.score_out = nullptr;
-        carve_scan(P, wsp, B, cap, m->H_idx);
-        wsp += topk_ws_one(B, cap, m->H_idx);
     }
+    carve_scan_workspace(sb, wsp, B, cap);
+    wsp += align_up(scan_workspace_bytes(sb.n, B, cap, m->H_idx));
     if (sb.n > 0) {
         rc = cuda_status(launch_index_topk(sb, st, ev ? ev + 3 : nullptr));
         if (rc) return rc;

@@ -15,10 +15,7 @@ struct ScanProblem {
     CacheView cache;
     const uint16_t* q_idx;  // bf16 [batch][H_idx][128]
     const float* w;         // fp32 [batch][H_idx]
-    uint8_t* qc;            // workspace: MXFP4 query codes [batch][H_idx][64]
-    uint8_t* qs;            // workspace: E8M0 query scales [batch][H_idx][4]
     float* scores;          // workspace: fp32 [batch][score_stride]
-    int64_t score_stride;
     int32_t* idx_out;       // [batch][K]
     float* score_out;       // nullable [batch][K]
 };
@@ -26,10 +23,18 @@ struct ScanProblem {
 constexpr int kMaxProblems = 64;
 struct ScanBatch {
     ScanProblem p[kMaxProblems];
+    uint8_t* qc;            // workspace: MXFP4 query codes [n][batch][H_idx][64]
+    uint8_t* qs;            // workspace: E8M0 query scales [n][batch][H_idx][4]
+    int64_t score_stride;   // entries per score row (>= every problem's capacity)
     int n;
     int H_idx;
     int K;
 };
+
+// Bytes of scan workspace for n problems.
+size_t scan_workspace_bytes(int n_problems, int batch, int max_entries, int H_idx);
+// Point sb.qc / sb.qs / every problem's scores into ws (sb.n must be set).
+void carve_scan_workspace(ScanBatch& sb, uint8_t* ws, int batch, int max_entries);
 
 // ev (nullable): events recorded after query quantisation, after the scan and
 // after Top-K (three cudaEvent_t).

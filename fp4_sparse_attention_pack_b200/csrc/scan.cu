@@ -65,6 +65,7 @@ __global__ void k_quant_queries(ScanBatch sb, int batch) {
     if (g >= batch * H * 4) return;
     const int blk = g & 3, bh = g >> 2;
     const uint16_t* src = P.q_idx + (int64_t)bh * DI + 32 * blk;
+    const int64_t qrow = (int64_t)prob * batch * H + bh;  // row of (problem, sequence, head)
     float v[32];
     float amax = 0.0f;
 #pragma unroll
@@ -72,11 +73,11 @@ __global__ void k_quant_queries(ScanBatch sb, int batch) {
         v[i] = bf16_bits_to_f32(src[i]);
         amax = fmaxf(amax, fabsf(v[i]));
     }
-    uint8_t* dst = P.qc + (int64_t)bh * ICB + 16 * blk;
+    uint8_t* dst = sb.qc + qrow * ICB + 16 * blk;
     if (amax == 0.0f) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) dst[i] = 0;
-        P.qs[(int64_t)bh * ISB + blk] = 0;
+        sb.qs[qrow * ISB + blk] = 0;
         return;
     }
     const int X = mx_shared_exp(amax);
@@ -85,7 +86,7 @@ __global__ void k_quant_queries(ScanBatch sb, int batch) {
     for (int i = 0; i < 16; ++i)
         dst[i] = (uint8_t)(e2m1_encode(__fmul_rn(v[2 * i], inv)) |
                            (e2m1_encode(__fmul_rn(v[2 * i + 1], inv)) << 4));
-    P.qs[(int64_t)bh * ISB + blk] = (uint8_t)(X + 127);
+    sb.qs[qrow * ISB + blk] = (uint8_t)(X + 127);
 }
 
 // ---- CUDA-core scan: thread per entry
@@ -99,13 +100,14 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_cuda(ScanBatch sb) {
     const int H = sb.H_idx;
     int32_t* qexp = sq + H * 32;
     float* wv = reinterpret_cast<float*>(qexp + H * 4);
+    const int64_t qrow0 = ((int64_t)prob * P.cache.batch + b) * H;
     for (int i = threadIdx.x; i < H * 32; i += blockDim.x) {
         const int h = i >> 5, wd = i & 31;
-        const uint8_t* qc = P.qc + ((int64_t)b * H + h) * ICB + 2 * wd;
+        const uint8_t* qc = sb.qc + (qrow0 + h) * ICB + 2 * wd;
         sq[i] = nib4_to_i8x4((uint32_t)qc[0] | ((uint32_t)qc[1] << 8));
     }
     for (int i = threadIdx.x; i < H * 4; i += blockDim.x)
-        qexp[i] = (int)P.qs[(int64_t)b * H * ISB + i] - 127;
+        qexp[i] = (int)sb.qs[qrow0 * ISB + i] - 127;
     for (int i = threadIdx.x; i < H; i += blockDim.x) wv[i] = P.w[(int64_t)b * H + i];
     __syncthreads();
 
@@ -149,12 +151,34 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_cuda(ScanBatch sb) {
         }
         score = fmaf(wv[h], fmaxf(dot, 0.0f), score);
     }
-    P.scores[(int64_t)b * P.score_stride + e] = score;
+    P.scores[(int64_t)b * sb.score_stride + e] = score;
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const ScanBatch& sb, cudaStream_t st);
+bool scan_mma_supported(const ScanBatch& sb);
+cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st);
+
+namespace {
+constexpr size_t kWsAlign = 256;
+inline size_t ws_align(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
+}  // namespace
+
+size_t scan_workspace_bytes(int n, int batch, int max_entries, int H_idx) {
+    return ws_align((size_t)n * batch * H_idx * ICB) + ws_align((size_t)n * batch * H_idx * ISB) +
+           ws_align((size_t)n * batch * max_entries * sizeof(float));
+}
+
+void carve_scan_workspace(ScanBatch& sb, uint8_t* ws, int batch, int max_entries) {
+    sb.qc = ws;
+    ws += ws_align((size_t)sb.n * batch * sb.H_idx * ICB);
+    sb.qs = ws;
+    ws += ws_align((size_t)sb.n * batch * sb.H_idx * ISB);
+    sb.score_stride = max_entries;
+    for (int i = 0; i < sb.n; ++i)
+        sb.p[i].scores = reinterpret_cast<float*>(ws) + (size_t)i * batch * max_entries;
+}
 
 cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t* ev) {
     const int batch = sb.p[0].cache.batch;
@@ -166,7 +190,11 @@ cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t*
         if (e != cudaSuccess) return e;
         if (ev) cudaEventRecord(ev[0], st);
     }
-    {
+    if (scan_mma_supported(sb)) {
+        cudaError_t e = launch_scan_mma(sb, st);
+        if (e != cudaSuccess) return e;
+        if (ev) cudaEventRecord(ev[1], st);
+    } else {
         int cap = 0;
         for (int i = 0; i < sb.n; ++i) cap = max(cap, sb.p[i].cache.max_pages * PAGE);
         dim3 grid((cap + kScanThreads - 1) / kScanThreads, batch, sb.n);

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kThreads) k_topk(ScanBatch sb) {
     const int b = blockIdx.x;
     const int K = sb.K;
     const int n = entries_of(P.cache, b);
-    const float* row = P.scores + (int64_t)b * P.score_stride;
+    const float* row = P.scores + (int64_t)b * sb.score_stride;
     int32_t* io = P.idx_out + (int64_t)b * K;
     float* so = P.score_out ? P.score_out + (int64_t)b * K : nullptr;
     const int tid = threadIdx.x;

@@ -299,10 +299,10 @@ def test_window_append_ring(csa):
 
 # ---------------------------------------------------------------- layer step
 
-@pytest.mark.parametrize("table_name", ["alternating", "pages"])
-def test_layer_step_parity(csa, table_name):
+@pytest.mark.parametrize("table_name,H_idx", [("alternating", 16), ("pages", 16), ("alternating", 64)])
+def test_layer_step_parity(csa, table_name, H_idx):
     table = W.schedule_alternating_40() if table_name == "alternating" else W.schedule_pages_40()
-    wl = W.Workload("small40", 7, 2, 601, table, 8, 16, 64, 3)
+    wl = W.Workload("small40", 7, 2, 601, table, 8, H_idx, 64, 3)
     dm = csa.engine.DecodeModel(wl, DEV, page_seed=21)
     dm.fill(chunk_tokens=256)
     rm = ref_model(wl)
