@@ -75,8 +75,14 @@ int csa2_pack_cache(const csa2_cache* cache, const void* x, int x_dtype, const f
     if (!x || !gates || !w_idx) return CSA2_ERR_INVALID_ARG;
     if (!a16(x) || !a16(w_idx)) return CSA2_ERR_ALIGN;
     if ((int64_t)T_new > (int64_t)cache->max_pages * PAGE * 2) return CSA2_ERR_INVALID_ARG;
-    return cuda_status(launch_pack(view_of(*cache), x, x_dtype == CSA2_DTYPE_F32, gates, w_idx, T_new,
-                                   (cudaStream_t)stream));
+    PackBatch pb;
+    std::memset(&pb, 0, sizeof(pb));
+    pb.n = 1;
+    pb.cache[0] = view_of(*cache);
+    pb.x[0] = x;
+    pb.gates[0] = gates;
+    pb.W[0] = w_idx;
+    return cuda_status(launch_pack(pb, x_dtype == CSA2_DTYPE_F32, T_new, (cudaStream_t)stream));
 }
 
 size_t csa2_index_topk_workspace(int batch, int max_entries, int H_idx, int K) {
@@ -135,7 +141,7 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const in
     if (batch < 1) return CSA2_ERR_INVALID_ARG;
     if (!a16(q) || !a16(out) || (ws && !a16(ws))) return CSA2_ERR_ALIGN;
     const size_t need = attn_workspace_bytes(1, batch, H, K);
-    if (!ws || ws_bytes < need) return CSA2_ERR_WORKSPACE;
+    if (need > 0 && (!ws || ws_bytes < need)) return CSA2_ERR_WORKSPACE;
     AttnBatch ab;
     std::memset(&ab, 0, sizeof(ab));
     ab.n = 1;
@@ -145,7 +151,7 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const in
     ab.scale = scale;
     const size_t units = need / ((D + 2) * sizeof(float));
     ab.part_o = static_cast<float*>(ws);
-    ab.part_ml = ab.part_o + units * D;
+    ab.part_ml = ab.part_o + units * D;  // CUDA-core layout; the tensor-core path re-derives it
     AttnProblem& P = ab.p[0];
     if (K > 0) P.cache = view_of(*cache);
     P.q = q;
@@ -283,10 +289,18 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
     if (ev) cudaEventRecord(ev[1], st);
 
     // (2) the Full layer of each source writes its new token into the cache
+    PackBatch pb;
+    std::memset(&pb, 0, sizeof(pb));
     for (int s = 0; s < m->n_sources; ++s) {
         if (!in->x_new[s]) continue;
-        rc = cuda_status(launch_pack(view_of(m->caches[s]), in->x_new[s], false, in->g_new[s],
-                                     m->w_idx[s], 1, st));
+        pb.cache[pb.n] = view_of(m->caches[s]);
+        pb.x[pb.n] = in->x_new[s];
+        pb.gates[pb.n] = in->g_new[s];
+        pb.W[pb.n] = m->w_idx[s];
+        ++pb.n;
+    }
+    if (pb.n > 0) {
+        rc = cuda_status(launch_pack(pb, false, 1, st));
         if (rc) return rc;
     }
     if (ev) cudaEventRecord(ev[2], st);

@@ -176,12 +176,20 @@ __global__ void k_window_append(WinAppend wa) {
 
 }  // namespace
 
+bool attn_mma_supported(const AttnBatch& ab);
+size_t attn_mma_workspace_bytes(int n_problems, int batch, int H, int Kmax);
+cudaError_t launch_attn_mma(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev);
+
 size_t attn_workspace_bytes(int n_problems, int batch, int H, int Kmax) {
+    if (H >= 1 && H <= 64) return attn_mma_workspace_bytes(n_problems, batch, H, Kmax);
     const size_t units = (size_t)n_problems * batch * n_splits(Kmax) * H;
     return units * D * sizeof(float) + units * 2 * sizeof(float);
 }
 
-cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev) {
+namespace {
+
+// CUDA-core path (heads beyond the tensor-core kernel's 64).
+cudaError_t launch_attn_cuda(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev) {
     const size_t smem = sizeof(float) * (kSplit * kStride + kWarps * D);
     static const bool attr_set = [smem] {
         cudaFuncSetAttribute(k_attn_split, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -198,6 +206,13 @@ cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t
     e = cudaGetLastError();
     if (e == cudaSuccess && ev) cudaEventRecord(ev[1], st);
     return e;
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev) {
+    if (attn_mma_supported(ab)) return launch_attn_mma(ab, st, ev);
+    return launch_attn_cuda(ab, st, ev);
 }
 
 cudaError_t launch_window_append(const WinAppend& wa, cudaStream_t st) {

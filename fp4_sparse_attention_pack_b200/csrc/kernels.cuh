@@ -5,9 +5,16 @@
 
 namespace csa2 {
 
-// ---- cache write
-cudaError_t launch_pack(const CacheView& c, const void* x, bool x_f32, const float* gates,
-                        const float* W, int T, cudaStream_t st);
+// ---- cache write: the same T new tokens per sequence for each listed source
+constexpr int kMaxPackSources = 8;
+struct PackBatch {
+    CacheView cache[kMaxPackSources];
+    const void* x[kMaxPackSources];      // [batch][T][512] bf16 or fp32
+    const float* gates[kMaxPackSources]; // [batch][T]
+    const float* W[kMaxPackSources];     // [512][128]
+    int n;
+};
+cudaError_t launch_pack(const PackBatch& pb, bool x_f32, int T, cudaStream_t st);
 
 // ---- indexer
 // One scan problem: one indexer query set over one cache, for all sequences.

@@ -42,12 +42,37 @@ __device__ __forceinline__ int new_entries(const CacheView& c, int b, int T, int
     return nn;
 }
 
+constexpr int kWc = 32;  // projection rows staged per step (32 x 128 fp32 = 16 KB)
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Rows [k*kWc, (k+1)*kWc) of W -> wb (128 threads, 8 x 16 B each).
+__device__ __forceinline__ void stage_w(float* wb, const float* W, int k) {
+    const float4* src = reinterpret_cast<const float4*>(W + (size_t)k * kWc * DI);
+    float4* dst = reinterpret_cast<float4*>(wb);
+#pragma unroll
+    for (int i = 0; i < kWc * DI / 4 / kThreads; ++i)
+        cp_async16(dst + threadIdx.x + i * kThreads, src + threadIdx.x + i * kThreads);
+    cp_async_commit();
+}
+
 template <bool kF32>
-__global__ void __launch_bounds__(kThreads) k_pack_entries(CacheView c, const void* x,
-                                                             const float* gates, const float* W,
-                                                             int T) {
-    extern __shared__ float deq[];  // [kEnt][512]
+__global__ void __launch_bounds__(kThreads) k_pack_entries(const __grid_constant__ PackBatch pb, int T) {
+    extern __shared__ float deq[];  // [kEnt][512], then W staging [2][kWc][128]
+    float* wbuf = deq + kEnt * D;
     __shared__ int s_page[kEnt];
+    const CacheView& c = pb.cache[blockIdx.z];
+    const void* x = pb.x[blockIdx.z];
+    const float* gates = pb.gates[blockIdx.z];
+    const float* W = pb.W[blockIdx.z];
     const int b = blockIdx.y;
     const int t = threadIdx.x;
     const int n0 = entries_of(c, b);
@@ -112,16 +137,33 @@ __global__ void __launch_bounds__(kThreads) k_pack_entries(CacheView c, const vo
     }
     __syncthreads();
 
-    // ---- phase 2: k[jj][o] = sum_c W[c][o] * deq[jj][c], fma order c = 0..511
+    // ---- phase 2: k[jj][o] = sum_c W[c][o] * deq[jj][c], fma order c = 0..511,
+    // W rows staged through shared memory (double-buffered cp.async)
     float acc[kEnt];
 #pragma unroll
     for (int jj = 0; jj < kEnt; ++jj) acc[jj] = 0.0f;
     const int o = t;
+    constexpr int kSteps = D / kWc;
+    stage_w(wbuf, W, 0);
 #pragma unroll 1
-    for (int ch = 0; ch < D; ++ch) {
-        const float w = __ldg(W + ch * DI + o);
+    for (int k = 0; k < kSteps; ++k) {
+        if (k + 1 < kSteps) {
+            stage_w(wbuf + ((k + 1) & 1) * kWc * DI, W, k + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const float* wb = wbuf + (k & 1) * kWc * DI;
+#pragma unroll 4
+        for (int cc = 0; cc < kWc; ++cc) {
+            const float w = wb[cc * DI + o];
+            const int ch = k * kWc + cc;
 #pragma unroll
-        for (int jj = 0; jj < kEnt; ++jj) acc[jj] = __fmaf_rn(w, deq[jj * D + ch], acc[jj]);
+            for (int jj = 0; jj < kEnt; ++jj)
+                if (jj < ne) acc[jj] = __fmaf_rn(w, deq[jj * D + ch], acc[jj]);
+        }
+        __syncthreads();
     }
 
     // ---- phase 3: MXFP4 per 32 channels (warp w = block w)
@@ -154,7 +196,10 @@ __global__ void __launch_bounds__(kThreads) k_pack_entries(CacheView c, const vo
 
 // Entry count and pending-slot update, after every entry was written.
 template <bool kF32>
-__global__ void k_pack_finalize(CacheView c, const void* x, const float* gates, int T) {
+__global__ void k_pack_finalize(const __grid_constant__ PackBatch pb, int T) {
+    const CacheView& c = pb.cache[blockIdx.y];
+    const void* x = pb.x[blockIdx.y];
+    const float* gates = pb.gates[blockIdx.y];
     const int b = blockIdx.x;
     const int n0 = entries_of(c, b);
     int pend;
@@ -179,30 +224,32 @@ __global__ void k_pack_finalize(CacheView c, const void* x, const float* gates, 
 
 }  // namespace
 
-cudaError_t launch_pack(const CacheView& c, const void* x, bool x_f32, const float* gates,
-                        const float* W, int T, cudaStream_t st) {
-    const int max_new = (c.ratio == 2) ? (T + 1) / 2 : T;
+cudaError_t launch_pack(const PackBatch& pb, bool x_f32, int T, cudaStream_t st) {
+    if (pb.n < 1 || T < 1) return cudaSuccess;
+    int max_new = (T + 1) / 2;
+    for (int i = 0; i < pb.n; ++i)
+        if (pb.cache[i].ratio == 1) max_new = T;
     const int chunks = (max_new + kEnt - 1) / kEnt;
-    if (chunks > 0) {
-        dim3 grid(chunks, c.batch);
-        const size_t smem = sizeof(float) * kEnt * D;
-        static const bool attr_set = [smem] {
-            cudaFuncSetAttribute(k_pack_entries<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            cudaFuncSetAttribute(k_pack_entries<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            return true;
-        }();
-        (void)attr_set;
-        if (x_f32)
-            k_pack_entries<true><<<grid, kThreads, smem, st>>>(c, x, gates, W, T);
-        else
-            k_pack_entries<false><<<grid, kThreads, smem, st>>>(c, x, gates, W, T);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
+    const int batch = pb.cache[0].batch;
+    const size_t smem = sizeof(float) * (kEnt * D + 2 * kWc * DI);
+    static const bool attr_set = [smem] {
+        cudaFuncSetAttribute(k_pack_entries<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(k_pack_entries<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        return true;
+    }();
+    (void)attr_set;
+    dim3 grid(chunks, batch, pb.n);
     if (x_f32)
-        k_pack_finalize<true><<<c.batch, 128, 0, st>>>(c, x, gates, T);
+        k_pack_entries<true><<<grid, kThreads, smem, st>>>(pb, T);
     else
-        k_pack_finalize<false><<<c.batch, 128, 0, st>>>(c, x, gates, T);
+        k_pack_entries<false><<<grid, kThreads, smem, st>>>(pb, T);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dim3 g2(batch, pb.n);
+    if (x_f32)
+        k_pack_finalize<true><<<g2, 128, 0, st>>>(pb, T);
+    else
+        k_pack_finalize<false><<<g2, 128, 0, st>>>(pb, T);
     return cudaGetLastError();
 }
 
