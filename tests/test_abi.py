@@ -61,8 +61,10 @@ def test_argument_checks_fail_before_launch(capi):
     assert lib.csa2_index_topk(ctypes.byref(c), ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 8,
                                ctypes.c_void_p(16), None, None, 0, None) == -6
     w = capi.csa2_window(16, 16, 1)
-    assert lib.csa2_sparse_attn(None, ctypes.c_void_p(16), 4, None, 0, ctypes.byref(w), 0.1,
+    # more than 64 heads take the CUDA-core path, which needs a workspace
+    assert lib.csa2_sparse_attn(None, ctypes.c_void_p(16), 100, None, 0, ctypes.byref(w), 0.1,
                                 ctypes.c_void_p(16), None, 0, None) == -6
+    assert capi.sparse_attn_workspace(1, 100, 0) > 0
     assert lib.csa2_sparse_attn(None, ctypes.c_void_p(16), 0, None, 0, ctypes.byref(w), 0.1,
                                 ctypes.c_void_p(16), None, 0, None) == -1
     assert capi.index_topk_workspace(2, 1024, 64, 512) > 2 * 1024 * 4
