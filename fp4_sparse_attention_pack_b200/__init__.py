@@ -151,3 +151,15 @@ def layer_step(model: csa2_model, step_in: csa2_step_in, step_out: csa2_step_out
     _ok(lib().csa2_layer_step(ctypes.byref(model), ctypes.byref(step_in), ctypes.byref(step_out),
                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
         "csa2_layer_step")
+
+
+def index_topk_noalloc(cache: csa2_cache, q_idx, w, K: int, idx_out, score_out=None, stream=None):
+    """csa2_index_topk without a workspace: for callers that cannot allocate
+    device memory (a fixed memory pool, no allocation on the decode path).  The
+    scratch is a fixed 8 MiB array inside the library; see include/csa2.h."""
+    f = lib().csa2_index_topk_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.POINTER(csa2_cache), _vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]
+    H_idx = q_idx.shape[1]
+    _ok(f(ctypes.byref(cache), _ptr(q_idx), _ptr(w), H_idx, K, _ptr(idx_out), _ptr(score_out),
+          _stream(stream)), "csa2_index_topk_noalloc")

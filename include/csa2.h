@@ -271,6 +271,34 @@ int csa2_layer_step(const csa2_model* model, const csa2_step_in* in, const csa2_
                     void* ws, size_t ws_bytes, csa2_stream stream);
 
 /*
+ * csa2_index_topk for callers that cannot allocate device memory.  (The pages
+ * have no counterpart; this is an interface of this library only.)
+ *
+ * Some callers cannot give the library a workspace: an engine whose device
+ * memory is a fixed pool reserved before decoding, with no allocation allowed
+ * on the decode path, or a plugin interface without a workspace argument.
+ * This call computes exactly what csa2_index_topk computes, with the same
+ * kernels and arguments, but keeps its scratch (quantised queries and one fp32
+ * score per entry) in a static array inside the library's device image:
+ * CSA2_NOALLOC_SCRATCH_BYTES (8 MiB) on every device that loads the library,
+ * held until the process exits.  The call itself allocates nothing.
+ *   - Size limit: the scratch needed, about batch * max_pages * 64 * 4 +
+ *     batch * H_idx * 68 bytes, must fit in 8 MiB; larger requests return
+ *     CSA2_ERR_UNSUPPORTED before anything is launched.
+ *   - Set-up: the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current).  Make that first call
+ *     before any stream capture.
+ *   - Sharing: every call uses the same array and leaves its contents behind
+ *     (nothing in it needs to start at zero).  Calls whose kernels overlap on
+ *     the GPU -- other streams or other host threads -- race; serialise them.
+ * Errors: as csa2_index_topk, plus CSA2_ERR_UNSUPPORTED for the size limit.
+ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (8u << 20)
+int csa2_index_topk_noalloc(const csa2_cache* cache, const uint16_t* q_idx, const float* w,
+                            int H_idx, int K, int32_t* idx_out, float* score_out,
+                            csa2_stream stream);
+
+/*
  * Measurement variant of csa2_layer_step: identical work, and in addition
  * records CUDA events on `stream` at the phase boundaries.  `events` is a host
  * array of CSA2_STEP_EVENTS cudaEvent_t handles (as void*) created by the caller
