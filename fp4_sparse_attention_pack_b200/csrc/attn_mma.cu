@@ -156,61 +156,85 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_mma(const __grid_constant_
     const uint32_t idesc_o = idesc_f16(128, kHp, 0, 1, 1);
 
     for (int t = t_begin; t < t_end && !timed_out; ++t) {
-        // ---- gather + dequantise 128 items (8 threads per item, one slab each)
-        for (int u = tid; u < kT * 8; u += kThreads) {
-            const int r = u >> 3, j = u & 7;
-            const int pos = t * kT + r;
-            uint8_t* slab = sm.items[j];
-            bool ok = false;
-            if (pos < K) {
-                const int e = P.idx[(int64_t)b * K + pos];
+        // ---- gather + dequantise 128 items: thread = slab j of items r0 + 32 i (i < 4).
+        // The dependent loads (index -> page -> bytes) of the four items are issued
+        // stage by stage so their latencies overlap.
+        {
+            const int j = tid & 7, r0 = tid >> 3;
+            int ent_i[4];
+            int64_t ent_row[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int pos = t * kT + r0 + 32 * i;
+                ent_i[i] = (pos < K) ? __ldg(P.idx + (int64_t)b * K + pos) : -1;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                ent_row[i] = -1;
+                const int e = ent_i[i];
                 if (e >= 0 && e < n) {
                     const int pg = page_of(P.cache, b, e);
-                    if (pg >= 0) {
-                        ok = true;
-                        const int64_t ent = (int64_t)pg * PAGE + (e % PAGE);
-                        const uint4* cs = reinterpret_cast<const uint4*>(P.cache.main_codes + ent * MCB + 32 * j);
-                        const uint4 c0 = cs[0], c1 = cs[1];
-                        const uint32_t sw = *reinterpret_cast<const uint32_t*>(P.cache.main_scales + ent * MSB + 4 * j);
-                        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    if (pg >= 0) ent_row[i] = (int64_t)pg * PAGE + (e % PAGE);
+                }
+            }
+            uint4 c0[4], c1[4];
+            uint32_t swd[4];
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {  // chunk c: channels 8c..8c+7, scale byte c/2
-                            const float s = e4m3_decode_pos((sw >> (8 * (c >> 1))) & 0xFFu);
-                            const __half2 s2 = __float2half2_rn(s);
-                            uint4 o;
-                            uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+            for (int i = 0; i < 4; ++i) {
+                if (ent_row[i] >= 0) {
+                    const uint4* cs = reinterpret_cast<const uint4*>(P.cache.main_codes + ent_row[i] * MCB + 32 * j);
+                    c0[i] = __ldg(cs);
+                    c1[i] = __ldg(cs + 1);
+                    swd[i] = __ldg(reinterpret_cast<const uint32_t*>(P.cache.main_scales + ent_row[i] * MSB + 4 * j));
+                }
+            }
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const __half2 v = __hmul2(sm.lut[(cw[c] >> (8 * k)) & 0xFFu], s2);
-                                os[k] = *reinterpret_cast<const uint32_t*>(&v);
-                            }
-                            *reinterpret_cast<uint4*>(slab + sw128(r, c)) = o;
+            for (int i = 0; i < 4; ++i) {
+                const int r = r0 + 32 * i;
+                const int pos = t * kT + r;
+                uint8_t* slab = sm.items[j];
+                bool ok = false;
+                if (ent_row[i] >= 0) {
+                    ok = true;
+                    const uint32_t cw[8] = {c0[i].x, c0[i].y, c0[i].z, c0[i].w, c1[i].x, c1[i].y, c1[i].z, c1[i].w};
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {  // chunk c: channels 8c..8c+7, scale byte c/2
+                        const __half2 s2 = __float2half2_rn(e4m3_decode_pos((swd[i] >> (8 * (c >> 1))) & 0xFFu));
+                        uint4 o;
+                        uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const __half2 v = __hmul2(sm.lut[(cw[c] >> (8 * k)) & 0xFFu], s2);
+                            os[k] = *reinterpret_cast<const uint32_t*>(&v);
                         }
+                        *reinterpret_cast<uint4*>(slab + sw128(r, c)) = o;
+                    }
+                } else if (pos >= K && pos - K < wlen) {
+                    ok = true;
+                    const uint4* src = reinterpret_cast<const uint4*>(P.win + ((int64_t)b * WIN + (pos - K)) * D + 64 * j);
+                    uint4 wv[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) wv[c] = __ldg(src + c);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t ws[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+                        uint4 o;
+                        uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const __half2 hv = __floats2half2_rn(__uint_as_float(ws[k] << 16),
+                                                                 __uint_as_float(ws[k] & 0xFFFF0000u));
+                            os[k] = *reinterpret_cast<const uint32_t*>(&hv);
+                        }
+                        *reinterpret_cast<uint4*>(slab + sw128(r, c)) = o;
                     }
                 }
-            } else if (pos - K < wlen) {
-                ok = true;
-                const uint4* src = reinterpret_cast<const uint4*>(P.win + ((int64_t)b * WIN + (pos - K)) * D + 64 * j);
+                if (!ok) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 w = src[c];
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                    uint4 o;
-                    uint32_t* os = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const __half2 hv = __floats2half2_rn(__uint_as_float(ws[k] << 16),
-                                                             __uint_as_float(ws[k] & 0xFFFF0000u));
-                        os[k] = *reinterpret_cast<const uint32_t*>(&hv);
-                    }
-                    *reinterpret_cast<uint4*>(slab + sw128(r, c)) = o;
+                    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(slab + sw128(r, c)) = make_uint4(0, 0, 0, 0);
                 }
+                if (j == 0) sm.valid[r] = ok;
             }
-            if (!ok) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(slab + sw128(r, c)) = make_uint4(0, 0, 0, 0);
-            }
-            if (j == 0) sm.valid[r] = ok;
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -276,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_mma(const __grid_constant_
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int h = 8 * c + 2 * k;
-                    const float p0 = ok ? expf(v[h] * ab.scale - sm.m_used[h]) : 0.0f;
-                    const float p1 = ok ? expf(v[h + 1] * ab.scale - sm.m_used[h + 1]) : 0.0f;
+                    const float p0 = ok ? __expf(v[h] * ab.scale - sm.m_used[h]) : 0.0f;
+                    const float p1 = ok ? __expf(v[h + 1] * ab.scale - sm.m_used[h + 1]) : 0.0f;
                     const __half2 hv = __floats2half2_rn(p0, p1);
                     const float2 back = __half22float2(hv);
                     v[h] = back.x;

@@ -132,72 +132,85 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            prefetch_tmap(&mp.queries);
-            const uint64_t pol_stream = policy_evict_first();
-            const uint64_t pol_keep = policy_evict_last();
-            uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0;
-            int issued[kStages];
-            uint32_t issued_par[kStages];
-            for (int s = 0; s < kStages; ++s) issued[s] = 0, issued_par[s] = 0;
-            for (int id = blockIdx.x; id < n_items && !aborted(sm); id += gridDim.x) {
-                Item it;
-                if (!item_at(sb, mp, id, it)) continue;
-                const ScanProblem& P = sb.p[it.p];
-                const CacheView& c = P.cache;
-                if (!mbar_wait(&sm.bempty[bslot], bphase ^ 1)) { raise_abort(sm, c.status); break; }
-                const int64_t qrow = ((int64_t)it.p * batch + it.b) * kHeads;
-                mbar_expect_tx(&sm.bfull[bslot], kHeads * 64 + kHeads * 4 + kHeads * 4);
-                tma_load_2d(sm.b[bslot], &mp.queries, 0, (int)qrow, &sm.bfull[bslot], pol_keep);
-                bulk_load(sm.sfb_raw[bslot], sb.qs + qrow * ISB, kHeads * 4, &sm.bfull[bslot], pol_keep);
-                bulk_load(sm.w[bslot], P.w + (int64_t)it.b * kHeads, kHeads * 4, &sm.bfull[bslot], pol_keep);
-                if (++bslot == 2) bslot = 0, bphase ^= 1;
-                const CUtensorMap* kmap = &mp.keys[mp.src_of[it.p]];
-                const int used_pages = (it.n + PAGE - 1) / PAGE;
-                bool stop = false;
-                for (int t = it.t0; t < it.t1; ++t) {
-                    if (!mbar_wait(&sm.empty[stage], sphase ^ 1)) { raise_abort(sm, c.status); stop = true; break; }
-                    int pg[2] = {-1, -1};
-                    uint32_t bytes = 0;
-                    for (int h = 0; h < 2; ++h) {
-                        const int li = 2 * t + h;  // logical page of this half tile
-                        if (li >= used_pages) continue;
-                        const int pp = c.page_table[(int64_t)it.b * c.max_pages + li];
-                        if (pp < 0 || pp >= c.num_pages) {
-                            atomicOr(c.status, CSA2_DEVERR_PAGE);
-                            continue;
-                        }
-                        pg[h] = pp;
-                        bytes += PAGE * ICB + PAGE * ISB;
-                    }
-                    if (bytes == 0) {
-                        mbar_arrive(&sm.full[stage]);
-                    } else {
-                        mbar_expect_tx(&sm.full[stage], bytes);
-                        for (int h = 0; h < 2; ++h) {
-                            if (pg[h] < 0) continue;
-                            tma_load_2d(sm.a[stage] + h * PAGE * ICB, kmap, 0, pg[h] * PAGE, &sm.full[stage],
-                                        pol_stream);
-                            bulk_load(sm.sfa_raw[stage] + h * PAGE * ISB, c.idx_scales + (int64_t)pg[h] * PAGE * ISB,
-                                      PAGE * ISB, &sm.full[stage], pol_stream);
-                        }
-                    }
-                    issued[stage] = 1;
-                    issued_par[stage] = sphase;
-                    if (++stage == kStages) stage = 0, sphase ^= 1;
-                }
-                if (stop) break;
+        // Lanes fetch the item's page ids (2 per tile, up to 32) in one round;
+        // lane 0 issues every copy.
+        const uint64_t pol_stream = policy_evict_first();
+        const uint64_t pol_keep = policy_evict_last();
+        if (lane == 0) prefetch_tmap(&mp.queries);
+        uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0;
+        int issued[kStages];
+        uint32_t issued_par[kStages];
+        for (int s = 0; s < kStages; ++s) issued[s] = 0, issued_par[s] = 0;
+        for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
+            Item it;
+            if (!item_at(sb, mp, id, it)) continue;
+            const ScanProblem& P = sb.p[it.p];
+            const CacheView& c = P.cache;
+            const int used_pages = (it.n + PAGE - 1) / PAGE;
+            const int li = 2 * it.t0 + lane;  // logical page this lane looks up
+            int my_pg = -1;
+            if (lane < 2 * (it.t1 - it.t0) && li < used_pages) {
+                const int pp = c.page_table[(int64_t)it.b * c.max_pages + li];
+                if (pp >= 0 && pp < c.num_pages)
+                    my_pg = pp;
+                else
+                    atomicOr(c.status, CSA2_DEVERR_PAGE);
             }
-            // never leave with copies in flight
+            bool stop = false;
+            if (lane == 0) {
+                if (!mbar_wait(&sm.bempty[bslot], bphase ^ 1)) {
+                    raise_abort(sm, c.status);
+                    stop = true;
+                } else {
+                    const int64_t qrow = ((int64_t)it.p * batch + it.b) * kHeads;
+                    mbar_expect_tx(&sm.bfull[bslot], kHeads * 64 + kHeads * 4 + kHeads * 4);
+                    tma_load_2d(sm.b[bslot], &mp.queries, 0, (int)qrow, &sm.bfull[bslot], pol_keep);
+                    bulk_load(sm.sfb_raw[bslot], sb.qs + qrow * ISB, kHeads * 4, &sm.bfull[bslot], pol_keep);
+                    bulk_load(sm.w[bslot], P.w + (int64_t)it.b * kHeads, kHeads * 4, &sm.bfull[bslot], pol_keep);
+                }
+            }
+            if (++bslot == 2) bslot = 0, bphase ^= 1;
+            const CUtensorMap* kmap = &mp.keys[mp.src_of[it.p]];
+            for (int t = it.t0; t < it.t1 && !__any_sync(0xffffffffu, stop); ++t) {
+                const int pg0 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0));
+                const int pg1 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0) + 1);
+                if (lane == 0) {
+                    if (!mbar_wait(&sm.empty[stage], sphase ^ 1)) {
+                        raise_abort(sm, c.status);
+                        stop = true;
+                    } else {
+                        const int pg[2] = {pg0, pg1};
+                        const uint32_t bytes = (pg0 >= 0 ? PAGE * (ICB + ISB) : 0) + (pg1 >= 0 ? PAGE * (ICB + ISB) : 0);
+                        if (bytes == 0) {
+                            mbar_arrive(&sm.full[stage]);
+                        } else {
+                            mbar_expect_tx(&sm.full[stage], bytes);
+                            for (int h = 0; h < 2; ++h) {
+                                if (pg[h] < 0) continue;
+                                tma_load_2d(sm.a[stage] + h * PAGE * ICB, kmap, 0, pg[h] * PAGE, &sm.full[stage],
+                                            pol_stream);
+                                bulk_load(sm.sfa_raw[stage] + h * PAGE * ISB,
+                                          c.idx_scales + (int64_t)pg[h] * PAGE * ISB, PAGE * ISB, &sm.full[stage],
+                                          pol_stream);
+                            }
+                        }
+                        issued[stage] = 1;
+                        issued_par[stage] = sphase;
+                    }
+                }
+                if (++stage == kStages) stage = 0, sphase ^= 1;
+            }
+            if (__any_sync(0xffffffffu, stop)) break;
+        }
+        // never leave with copies in flight
+        if (lane == 0)
             for (int s = 0; s < kStages; ++s)
                 if (issued[s]) (void)mbar_wait(&sm.full[s], issued_par[s]);
-        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0, acc = 0, aphase = 0;
         const uint32_t idesc_lo = idesc_mxf4(kHeads, 0, 0);
         const uint32_t idesc_hi = idesc_mxf4(kHeads, 2, 2);
-        bool issued_any = false;
         for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
             Item it;
             if (!item_at(sb, mp, id, it)) continue;
@@ -239,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tc_mma_mxf4(d, adesc + 2, bdesc + 2, idesc_hi, sfa, sfb, 1u);
                     tc_commit(&sm.empty[stage]);
                     tc_commit(&sm.tfull[acc]);
-                    issued_any = true;
                 }
                 __syncwarp();
                 if (++stage == kStages) stage = 0, sphase ^= 1;
@@ -256,7 +268,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             tc_commit(&sm.drained);
             (void)mbar_wait(&sm.drained, 0);
         }
-        (void)issued_any;
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
@@ -279,9 +290,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.tempty[acc]);
-                float s = 0.0f;
+                float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent chains
 #pragma unroll
-                for (int h = 0; h < kHeads; ++h) s = fmaf(w[h], fmaxf(v[h], 0.0f), s);
+                for (int h = 0; h < kHeads; h += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(w + h);
+                    part[0] = fmaf(w4.x, fmaxf(v[h], 0.0f), part[0]);
+                    part[1] = fmaf(w4.y, fmaxf(v[h + 1], 0.0f), part[1]);
+                    part[2] = fmaf(w4.z, fmaxf(v[h + 2], 0.0f), part[2]);
+                    part[3] = fmaf(w4.w, fmaxf(v[h + 3], 0.0f), part[3]);
+                }
+                const float s = (part[0] + part[1]) + (part[2] + part[3]);
                 const int e = t * kTile + row;
                 if (e < it.n) out[e] = s;
                 acc ^= 1;

@@ -1,11 +1,21 @@
-// Per-sequence Top-K of the indexer scores: block-level radix select.
+// Per-sequence Top-K of the indexer scores ("n'en garde que les 512 meilleures").
 //
-// Scores map to order-preserving uint32 keys.  Three MSB-first passes with
-// 11/11/10-bit digits find the key T of the K-th largest score and how many
-// elements equal to T are still needed; a final pass compacts, in index order,
-// every element with key > T and the first `need` elements with key == T
-// (equal scores: lower index first).  The output is therefore sorted by index.
-// One CTA of 1024 threads per (problem, sequence).
+// Scores map to order-preserving uint32 keys; the K largest are kept, equal
+// scores lower index first, and written in increasing index order.
+//
+// One CTA of 1024 threads per (problem, sequence):
+//   1. Threshold guess: 2,048 strided samples of the row; an exact radix select
+//      in shared memory finds the sample key ranked ~2K * 2048 / n, so that
+//      about 2K of the n scores lie at or above it.
+//   2. One pass over the row compacts every score at or above the guess, in
+//      index order, into shared memory (at most kCap).  If fewer than K or more
+//      than kCap qualify, the CTA falls back to an exact radix select over the
+//      whole row (two or more passes), so the result never depends on the guess.
+//   3. Exact radix select among the candidates (8-bit digits, warp-aggregated
+//      shared-memory histograms), then an ordered compaction of the keys above
+//      the K-th key plus the first `need` keys equal to it.
+// A key equal to the K-th largest is >= the guess whenever >= K keys are, so
+// every member of the Top-K (ties included) is among the candidates.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -14,6 +24,17 @@ namespace csa2 {
 namespace {
 
 constexpr int kThreads = 1024;
+constexpr int kSamples = 2048;
+constexpr int kCap = 12288;
+
+struct TopkSmem {
+    uint32_t key[kCap];
+    int32_t idx[kCap];
+    int hist[256];
+    int warp_tot[33];
+    int sel[2];
+    int flag;
+};
 
 // Exclusive prefix sum of one int per thread over the block; returns the total.
 __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* excl) {
@@ -34,8 +55,8 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* excl) {
             int y = __shfl_up_sync(0xffffffffu, u, o);
             if (lane >= o) u += y;
         }
-        s_warp[lane] = u - t;       // exclusive warp offsets
-        if (lane == 31) s_warp[32] = u;  // total
+        s_warp[lane] = u - t;
+        if (lane == 31) s_warp[32] = u;
     }
     __syncthreads();
     *excl = s_warp[wid] + x - v;
@@ -44,10 +65,81 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* excl) {
     return total;
 }
 
-__global__ void __launch_bounds__(kThreads) k_topk(ScanBatch sb) {
-    __shared__ int hist[2048];
-    __shared__ int s_warp[33];
-    __shared__ int s_sel[2];
+// Add one to hist[d] for every active lane with d < 256, one atomic per distinct d.
+__device__ __forceinline__ void hist_add(int* hist, uint32_t d) {
+    const unsigned act = __activemask();
+    const unsigned same = __match_any_sync(act, d);
+    if (d < 256 && (threadIdx.x & 31) == (__ffs(same) - 1)) atomicAdd(&hist[d], __popc(same));
+}
+
+// Exact radix select: the k-th largest key among key(i), i < cnt (k <= cnt), and
+// how many keys equal to it belong to the top k.  8-bit digits, MSB first.
+template <class KeyAt>
+__device__ void radix_select(KeyAt key_at, int cnt, int k, TopkSmem& sm, uint32_t* kth, int* need) {
+    uint32_t prefix = 0, mask = 0;
+    int remaining = k;
+    const int tid = threadIdx.x;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int sh = 24 - 8 * pass;
+        if (tid < 256) sm.hist[tid] = 0;
+        __syncthreads();
+        for (int i0 = 0; i0 < cnt; i0 += kThreads) {
+            const int i = i0 + tid;
+            uint32_t d = 256;
+            if (i < cnt) {
+                const uint32_t kk = key_at(i);
+                if ((kk & mask) == prefix) d = (kk >> sh) & 255u;
+            }
+            hist_add(sm.hist, d);
+        }
+        __syncthreads();
+        // bins in decreasing digit order: thread t owns digit 255 - t
+        const int c = tid < 256 ? sm.hist[255 - tid] : 0;
+        int above;
+        block_excl_scan(c, sm.warp_tot, &above);
+        if (tid < 256 && above < remaining && above + c >= remaining) {
+            sm.sel[0] = 255 - tid;
+            sm.sel[1] = remaining - above;
+        }
+        __syncthreads();
+        prefix |= (uint32_t)sm.sel[0] << sh;
+        mask |= 255u << sh;
+        remaining = sm.sel[1];
+        __syncthreads();
+    }
+    *kth = prefix;
+    *need = remaining;
+}
+
+// Ordered compaction of the Top-K: keys above kth, then (in index order) the
+// first `need` keys equal to it.  Writes out positions [0, K).
+template <class KeyAt, class IdxAt>
+__device__ void emit_topk(KeyAt key_at, IdxAt idx_at, int cnt, uint32_t kth, int need, int K,
+                          TopkSmem& sm, int32_t* io, float* so) {
+    int base = 0, eq_seen = 0;
+    for (int i0 = 0; i0 < cnt; i0 += kThreads) {
+        const int i = i0 + threadIdx.x;
+        const uint32_t kk = i < cnt ? key_at(i) : 0u;
+        const int gt = (i < cnt) && (kk > kth);
+        const int eq = (i < cnt) && (kk == kth);
+        int eq_rank;
+        const int eq_tot = block_excl_scan(eq, sm.warp_tot, &eq_rank);
+        const int take = gt || (eq && (eq_seen + eq_rank) < need);
+        int pos;
+        const int take_tot = block_excl_scan(take, sm.warp_tot, &pos);
+        if (take && base + pos < K) {
+            io[base + pos] = idx_at(i);
+            if (so) so[base + pos] = order_key_f32(kk);
+        }
+        base += take_tot;
+        eq_seen += eq_tot;
+        if (base >= K) break;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanBatch sb) {
+    extern __shared__ uint8_t smem_raw[];
+    TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
     const ScanProblem& P = sb.p[blockIdx.y];
     const int b = blockIdx.x;
     const int K = sb.K;
@@ -65,62 +157,50 @@ __global__ void __launch_bounds__(kThreads) k_topk(ScanBatch sb) {
         return;
     }
 
-    uint32_t prefix = 0, mask = 0;
-    int remaining = K;
-    const int shifts[3] = {21, 10, 0};
-    const int widths[3] = {11, 11, 10};
-    for (int pass = 0; pass < 3; ++pass) {
-        const int sh = shifts[pass], nb = 1 << widths[pass];
-        for (int i = tid; i < 2048; i += kThreads) hist[i] = 0;
+    // 1. threshold guess from strided samples (all scores qualify when they fit)
+    uint32_t guess = 0;
+    if (n > kCap) {
+        for (int i = tid; i < kSamples; i += kThreads)
+            sm.key[i] = f32_order_key(row[(int64_t)i * n / kSamples]);
         __syncthreads();
-        for (int i = tid; i < n; i += kThreads) {
-            const uint32_t k = f32_order_key(row[i]);
-            if ((k & mask) == prefix) atomicAdd(&hist[(k >> sh) & (nb - 1)], 1);
-        }
-        __syncthreads();
-        // suffix counts: thread t owns bins [2t, 2t+1]; scan from the top bin
-        const int t_hi = kThreads - 1 - tid;  // reversed owner so the scan runs top-down
-        int c0 = 0, c1 = 0;
-        if (2 * t_hi + 1 < nb) c1 = hist[2 * t_hi + 1];
-        if (2 * t_hi < nb) c0 = hist[2 * t_hi];
-        int above;
-        block_excl_scan(c0 + c1, s_warp, &above);  // count in bins above 2*t_hi+1
-        // the digit where the running count from the top reaches `remaining`
-        if (2 * t_hi + 1 < nb && above < remaining && above + c1 >= remaining) {
-            s_sel[0] = 2 * t_hi + 1;
-            s_sel[1] = remaining - above;
-        } else if (2 * t_hi < nb && above + c1 < remaining && above + c1 + c0 >= remaining) {
-            s_sel[0] = 2 * t_hi;
-            s_sel[1] = remaining - above - c1;
-        }
-        __syncthreads();
-        prefix |= (uint32_t)s_sel[0] << sh;
-        mask |= (uint32_t)(nb - 1) << sh;
-        remaining = s_sel[1];
-        __syncthreads();
+        const int rank = min(kSamples, (int)(((int64_t)2 * K * kSamples + n - 1) / n) + 16);
+        int unused;
+        radix_select([&](int i) { return sm.key[i]; }, kSamples, rank, sm, &guess, &unused);
     }
-    const uint32_t T = prefix;
-    const int need_eq = remaining;  // elements equal to T still to take
 
-    int base = 0, eq_seen = 0;
-    for (int start = 0; start < n; start += kThreads) {
-        const int i = start + tid;
-        const float f = i < n ? row[i] : 0.0f;
-        const uint32_t k = f32_order_key(f);
-        const int gt = (i < n) && (k > T);
-        const int eq = (i < n) && (k == T);
-        int eq_rank;
-        const int eq_tot = block_excl_scan(eq, s_warp, &eq_rank);
-        const int take = gt || (eq && (eq_seen + eq_rank) < need_eq);
+    // 2. one pass: ordered compaction of the scores at or above the guess
+    int cnt = 0;
+    bool fits = true;
+    for (int i0 = 0; i0 < n; i0 += kThreads) {
+        const int i = i0 + tid;
+        const uint32_t kk = i < n ? f32_order_key(row[i]) : 0u;
+        const int c = (i < n) && (kk >= guess);
         int pos;
-        const int take_tot = block_excl_scan(take, s_warp, &pos);
-        if (take && base + pos < K) {
-            io[base + pos] = i;
-            if (so) so[base + pos] = f;
+        const int tot = block_excl_scan(c, sm.warp_tot, &pos);
+        if (c && cnt + pos < kCap) {
+            sm.key[cnt + pos] = kk;
+            sm.idx[cnt + pos] = i;
         }
-        base += take_tot;
-        eq_seen += eq_tot;
-        if (base >= K) break;
+        cnt += tot;
+        if (cnt > kCap) {
+            fits = false;
+            break;
+        }
+    }
+    __syncthreads();
+
+    uint32_t kth;
+    int need;
+    if (fits && cnt >= K) {
+        // 3. exact selection among the candidates (already in index order)
+        radix_select([&](int i) { return sm.key[i]; }, cnt, K, sm, &kth, &need);
+        emit_topk([&](int i) { return sm.key[i]; }, [&](int i) { return sm.idx[i]; }, cnt, kth, need, K, sm,
+                  io, so);
+    } else {
+        // the guess failed: exact radix select over the whole row
+        auto gkey = [&](int i) { return f32_order_key(row[i]); };
+        radix_select(gkey, n, K, sm, &kth, &need);
+        emit_topk(gkey, [](int i) { return i; }, n, kth, need, K, sm, io, so);
     }
 }
 
@@ -128,8 +208,14 @@ __global__ void __launch_bounds__(kThreads) k_topk(ScanBatch sb) {
 
 cudaError_t launch_topk(const ScanBatch& sb, cudaStream_t st) {
     const int batch = sb.p[0].cache.batch;
+    const size_t smem = sizeof(TopkSmem);
+    static const bool attr = [smem] {
+        cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        return true;
+    }();
+    (void)attr;
     dim3 grid(batch, sb.n);
-    k_topk<<<grid, kThreads, 0, st>>>(sb);
+    k_topk<<<grid, kThreads, smem, st>>>(sb);
     return cudaGetLastError();
 }
 

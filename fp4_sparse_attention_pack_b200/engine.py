@@ -149,6 +149,25 @@ class DecodeModel:
         for l in range(self.L):
             self.load_window(l, T)
 
+    def append_turn(self, chunk_tokens: int = 8192):
+        """Agent turn of the prefix-cache workload: append tokens [T, T + append)
+        of every source (paged cache write) and refresh the windows to T + append."""
+        wl, B = self.wl, self.wl.B
+        if wl.append <= 0:
+            return
+        for s in range(self.S):
+            kx = synth.key(wl.seed, synth.TID_SRC_X, s)
+            kg = synth.key(wl.seed, synth.TID_SRC_G, s)
+            for t0 in range(wl.T, wl.T + wl.append, chunk_tokens):
+                n = min(chunk_tokens, wl.T + wl.append - t0)
+                x = torch.empty(B, n, D, dtype=torch.bfloat16, device=self.dev)
+                g = torch.empty(B, n, dtype=torch.float32, device=self.dev)
+                synth.dev_normal_bf16_rows(x, kx, t0 * D, synth.TSTRIDE * D, B, n * D, self.chan[s])
+                synth.dev_normal_f32_rows(g, kg, t0, synth.TSTRIDE, B, n)
+                pack_cache(self.caches[s].desc, x, g, self.W[s])
+        for l in range(self.L):
+            self.load_window(l, wl.T + wl.append)
+
     def load_window(self, l: int, T: int):
         wl, B = self.wl, self.wl.B
         n = min(T, WIN)

@@ -1,0 +1,153 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py times.
+
+The device fills every cache with the seeded recipe (device generator) and runs
+decode steps through csa2_layer_step; the oracle rebuilds only sampled sequences
+from the host generator and checks them: packed caches byte for byte, Top-K sets
+(tie band), attention outputs (2e-3).  The oracle never sees device data.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle
+from fp4_sparse_attention_pack_b200 import workloads as W
+
+from .oracle_models import ref_cache, ref_window
+from .parity import ATTN_REL, attn_rel_err, check_topk
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def engine():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from fp4_sparse_attention_pack_b200 import _build
+    _build.build()
+    from fp4_sparse_attention_pack_b200 import engine as e
+    return e
+
+
+def _check_cache(dc, rc, b_dev, n, ranges=None):
+    ranges = ranges or [(0, n)]
+    for lo, hi in ranges:
+        mc, ms, kc, ks = dc.logical(b_dev, lo, hi)
+        assert np.array_equal(ms, rc.ms[0, lo:hi]) and np.array_equal(mc, rc.mc[0, lo:hi]), (lo, hi)
+        assert np.array_equal(ks, rc.ks[0, lo:hi]) and np.array_equal(kc, rc.kc[0, lo:hi]), (lo, hi)
+
+
+def _check_layer(dm, wl, l, b, st, rcache, T_now):
+    """Top-K and attention of layer l, sequence b after step st, against the oracle."""
+    t = wl.table
+    m = t.mode[l]
+    gidx = dm.idx.cpu().numpy()
+    ties = 0
+    if m in (W.FULL, W.REINDEX):
+        sc = rcache.scores(0, W.query_idx(wl, l, st)[b], W.head_weights(wl, l, st)[b])
+        ties = check_topk(gidx[l, b], sc, wl.K)
+    ring, cnt = ref_window(wl, l, b, T_now)
+    if m == W.SWA_ONLY:
+        items = oracle.attention_items(np.zeros((1, 256), np.uint8), np.zeros((1, 32), np.uint8), 0,
+                                       np.zeros(0, np.int32), ring, min(cnt, 128))
+    else:
+        src_l = t.idx_src[l] if m == W.REUSE else l
+        items = oracle.attention_items(rcache.mc[0], rcache.ms[0], int(rcache.n[0]), gidx[src_l, b], ring,
+                                       min(cnt, 128))
+    ref = oracle.attention(W.query(wl, l, st)[b], items, wl.scale)
+    err = attn_rel_err(dm.out[l, b].cpu().numpy(), ref)
+    assert err <= ATTN_REL, (l, b, err)
+    return ties
+
+
+def test_config1_full_size(engine):
+    wl = W.WORKLOADS[1]  # 1 Full layer, B 8, 65,536 tokens, 64 + 64 heads, K 512
+    dm = engine.DecodeModel(wl, "cuda", page_seed=41, steps_capacity=4)
+    dm.fill()
+    dm.gen_step_inputs(0)
+    dm.step()
+    torch.cuda.synchronize()
+    assert dm.status_bits() == 0
+    for b in (0, 7):
+        rc = ref_cache(wl, 0, [b], wl.T + 1, cap=wl.T // 2 + 64)
+        _check_cache(dm.caches[0], rc, b, wl.T // 2)
+        _check_layer(dm, wl, 0, b, 0, rc, wl.T + 1)
+
+
+def test_config2_full_size(engine):
+    wl = W.WORKLOADS[2]  # 40 layers, B 16, 131,072 tokens, 23 scans per step
+    dm = engine.DecodeModel(wl, "cuda", steps_capacity=4)
+    dm.fill()
+    for st in range(2):  # the second step completes a ratio-2 group in every source
+        dm.gen_step_inputs(st)
+        dm.step()
+    torch.cuda.synchronize()
+    assert dm.status_bits() == 0
+    T_now = wl.T + 2
+    b = 5
+    for s, layers in ((3, (20, 21, 22, 39)), (0, (2, 3, 4))):
+        rc = ref_cache(wl, s, [b], T_now, cap=T_now // 2 + 64)
+        assert dm.caches[s].n_entries[b].item() == rc.n[0] == T_now // 2
+        _check_cache(dm.caches[s], rc, b, int(rc.n[0]), ranges=[(0, 4096), (int(rc.n[0]) - 4096, int(rc.n[0]))])
+        for l in layers:
+            _check_layer(dm, wl, l, b, 1, rc, T_now)
+    _check_layer(dm, wl, 0, b, 1, None, T_now)  # window-only layer
+
+
+def test_config3_full_size_outliers(engine):
+    wl = W.WORKLOADS[3]  # B 4, 1,048,576 tokens, K 1024, outlier channels
+    dm = engine.DecodeModel(wl, "cuda", steps_capacity=2)
+    dm.fill(chunk_tokens=16384)
+    dm.gen_step_inputs(0)
+    dm.step()
+    torch.cuda.synchronize()
+    assert dm.status_bits() == 0
+    b = 2
+    rc = ref_cache(wl, 0, [b], wl.T + 1, cap=wl.T // 2 + 64)
+    n = wl.T // 2
+    _check_cache(dm.caches[0], rc, b, n, ranges=[(0, 8192), (n // 2, n // 2 + 8192), (n - 8192, n)])
+    _check_layer(dm, wl, 0, b, 0, rc, wl.T + 1)
+
+
+def test_config4_paged_append_then_decode(engine):
+    wl = W.WORKLOADS[4]  # B 16, 262,144 cached + 8,192 appended tokens, paged, 40 layers
+    steps = 3
+    dm = engine.DecodeModel(wl, "cuda", page_seed=7, steps_capacity=steps)
+    dm.fill()
+    dm.append_turn()
+    torch.cuda.synchronize()
+    b, s = 11, 1
+    T1 = wl.T + wl.append
+    rc = ref_cache(wl, s, [b], T1, cap=T1 // 2 + 64)
+    assert dm.caches[s].n_entries[b].item() == T1 // 2
+    _check_cache(dm.caches[s], rc, b, T1 // 2, ranges=[(wl.T // 2, T1 // 2)])  # the appended turn
+    for st in range(steps):
+        dm.gen_step_inputs(st)
+        dm.step()
+    torch.cuda.synchronize()
+    assert dm.status_bits() == 0
+    T_now = T1 + steps
+    rc = ref_cache(wl, s, [b], T_now, cap=T_now // 2 + 64)
+    _check_cache(dm.caches[s], rc, b, int(rc.n[0]), ranges=[(int(rc.n[0]) - 64, int(rc.n[0]))])
+    for l in (8, 9, 10):
+        _check_layer(dm, wl, l, b, steps - 1, rc, T_now)
+
+
+def test_topk_all_equal_scores_takes_lowest_indices(engine):
+    # more equal scores than the candidate buffer holds: the full-row fallback
+    import fp4_sparse_attention_pack_b200 as csa
+    wl = W.small(W.WORKLOADS[1], B=1, T=2 * 20000)
+    dc = engine.DecodeModel  # noqa: F841 (engine module import check)
+    from fp4_sparse_attention_pack_b200.engine import DeviceCache
+    cache = DeviceCache(1, 20000 // 64 + 2, 2, "cuda")
+    tok = np.repeat(W.tokens(wl, 0, 0, 0, 1), 2 * 20000, axis=0)[None]
+    x = torch.from_numpy(tok.view(np.int16)).cuda().view(torch.bfloat16)
+    g = torch.zeros(1, 2 * 20000, device="cuda")
+    csa.pack_cache(cache.desc, x, g, torch.from_numpy(W.w_idx(wl, 0)).cuda())
+    q = torch.from_numpy(W.query_idx(wl, 0, 0).view(np.int16)).cuda().view(torch.bfloat16)
+    w = torch.from_numpy(W.head_weights(wl, 0, 0)).cuda()
+    idx = torch.empty(1, 512, dtype=torch.int32, device="cuda")
+    ws = torch.empty(csa.index_topk_workspace(1, cache.max_pages * 64, 64, 512), dtype=torch.uint8, device="cuda")
+    csa.index_topk(cache.desc, q, w, 512, idx, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx[0].cpu().numpy(), np.arange(512))
