@@ -16,10 +16,18 @@
 // a tile's maximum exceeds it by more than 8 (so p <= e^8 fits fp16), which
 // makes the O rescale (TMEM load, scale, store) rare.  Heads are padded to 64.
 //
-// CTA = 256 threads, one unit (problem, sequence, split of tiles) per CTA.  All
-// warps gather + dequantise a tile (8 threads per item, one 64-channel slab
-// each); thread 0 issues the MMAs; warps 0-3 (one TMEM lane quadrant each) run
-// the softmax; all 8 warps rescale / write O.
+// CTA = 256 threads, one unit (problem, sequence, split of tiles) per CTA.
+// Gather: the unit's selected entries and window are prefetched into L2 first;
+// window rows arrive by TMA (a 3-D tensor map per window, 128-byte swizzle, one
+// box per slab, so they land directly in the slab layout and are converted
+// bf16 -> fp16 in place); cache entries are loaded with 16-byte loads (eight
+// lanes per entry row) and dequantised in registers, the chunk order staggered
+// per lane so the swizzled stores are free of bank conflicts.  Thread 0 issues the MMAs; all eight
+// warps run the softmax (two per TMEM lane quadrant, 32 heads each) and
+// rescale / write O.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <cstring>
 
@@ -43,36 +51,71 @@ constexpr uint32_t kColS = 0;      // S^T: 64 columns
 constexpr uint32_t kColO = 64;     // O^T: 4 x 64 columns
 constexpr float kRescaleGap = 8.0f;
 
+struct AttnMaps {
+    CUtensorMap win[kMaxProblems];  // window [batch][128][512] bf16, box 64 x 128 x 1, SW128
+};
+
 struct __align__(1024) Smem {
     uint8_t items[8][kT * 128];    // 8 slabs x 128 rows x 128 B (SW128)
     uint8_t q[8][kHp * 128];       // 8 slabs x 64 rows x 128 B (SW128)
     uint8_t p[kT * 128];           // P^T: 128 item rows x 64 heads fp16 (SW128)
-    __half2 lut[256];              // code byte -> two E2M1 values
-    float red[4][kHp];             // per-warp partial max / sum
+    float red[4][kHp];             // per-quadrant partial max / sum
     float m_used[kHp];
     float l[kHp];
     float alpha[kHp];
-    int valid[kT];
-    uint64_t bar;
+    int kind[2][kT];               // per tile buffer: 0 empty, 1 cache entry, 2 window token
+    int64_t src_row[2][kT];        // entry row in the pools
+    int n_entries[2];
+    int has_window[2];
+    uint64_t bar;                  // MMA completion
+    uint64_t wbar;                 // window TMA
     uint32_t tmem_base;
 };
-
-__device__ __forceinline__ float e2m1_mag(uint32_t m) {
-    return m < 2 ? 0.5f * (float)m : __uint_as_float(((126u + (m >> 1)) << 23) | ((m & 1u) << 22));
-}
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory beyond the 227 KB per-block limit");
 
 // Byte offset of 16-byte chunk c of row r inside a 128B-swizzled slab.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
-// Reduce-scatter over the warp: v[64] per lane -> lane l holds the reduction of
-// heads 2l and 2l+1 over the 32 lanes in v[0], v[1].
-template <bool kMax>
-__device__ __forceinline__ void warp_reduce_scatter64(float (&v)[64]) {
+// Convert the 8 bf16 chunks (64 channels) of row r of a slab to fp16 in place
+// (exact for values in fp16's normal range).
+__device__ __forceinline__ void bf16_row_to_f16(uint8_t* slab, int r) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4* ptr = reinterpret_cast<uint4*>(slab + sw128(r, c));
+        const uint4 w = *ptr;
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        uint4 o;
+        uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const __half2 hv = __floats2half2_rn(__uint_as_float(ws[k] << 16), __uint_as_float(ws[k] & 0xFFFF0000u));
+            os[k] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        *ptr = o;
+    }
+}
+
+// Two E2M1 codes (one byte, channel 2i in the low nibble) -> f16x2 (low half first).
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(out) : "r"(byte));
+    return out;
+}
+
+__device__ __forceinline__ void zero_row(uint8_t* slab, int r) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(slab + sw128(r, c)) = make_uint4(0, 0, 0, 0);
+}
+
+// Reduce-scatter over the warp: v[N] per lane (N = 32 or 64) -> lane l holds the
+// reduction over the 32 lanes of element N/32 * l + i in v[i], i < N/32.
+template <bool kMax, int N>
+__device__ __forceinline__ void warp_reduce_scatter(float (&v)[N]) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int step = 0; step < 5; ++step) {
         const int o = 16 >> step;
-        const int half = 32 >> step;
+        const int half = (N / 2) >> step;
         const bool upper = (lane & o) != 0;
 #pragma unroll
         for (int i = 0; i < half; ++i) {
@@ -84,8 +127,9 @@ __device__ __forceinline__ void warp_reduce_scatter64(float (&v)[64]) {
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_attn_mma(const __grid_constant__ AttnBatch ab, int splits,
-                                                           int tiles_per_split) {
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_mma(const __grid_constant__ AttnBatch ab, const __grid_constant__ AttnMaps maps, int splits,
+               int tiles_per_split) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -103,155 +147,195 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_mma(const __grid_constant_
 
     if (tid == 0) {
         mbar_init(&sm.bar, 1);
+        mbar_init(&sm.wbar, 1);
+        sm.n_entries[0] = sm.n_entries[1] = 0;
+        sm.has_window[0] = sm.has_window[1] = 0;
         fence_mbar_init();
+        prefetch_tmap(&maps.win[prob]);
     }
     if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
-    for (int i = tid; i < 256; i += kThreads) {
-        const uint32_t lo = i & 15u, hi = i >> 4;
-        const float a = (lo & 8u) ? -e2m1_mag(lo & 7u) : e2m1_mag(lo & 7u);
-        const float c = (hi & 8u) ? -e2m1_mag(hi & 7u) : e2m1_mag(hi & 7u);
-        sm.lut[i] = __floats2half2_rn(a, c);
-    }
     if (tid < kHp) {
         sm.m_used[tid] = -INFINITY;
         sm.l[tid] = 0.0f;
     }
-    // Q -> fp16 slabs (rows >= H are zero)
-    for (int u = tid; u < kHp * 8; u += kThreads) {
-        const int h = u >> 3, j = u & 7;
-        uint8_t* slab = sm.q[j];
-        if (h < H) {
-            const uint4* src = reinterpret_cast<const uint4*>(P.q + ((int64_t)b * H + h) * D + 64 * j);
+    // Q -> fp16 slabs (rows >= H are zero): cp.async in place, then convert.
+    {
+        const int j = warp;
+        for (int h = lane; h < kHp; h += 32) {
+            if (h < H) {
+                const uint16_t* src = P.q + ((int64_t)b * H + h) * D + 64 * j;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 w = src[c];
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                uint4 o;
-                uint32_t* os = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const __half2 hv = __floats2half2_rn(__uint_as_float(ws[k] << 16),
-                                                         __uint_as_float(ws[k] & 0xFFFF0000u));
-                    os[k] = *reinterpret_cast<const uint32_t*>(&hv);
-                }
-                *reinterpret_cast<uint4*>(slab + sw128(h, c)) = o;
+                for (int c = 0; c < 8; ++c) cp_async16(sm.q[j] + sw128(h, c), src + 8 * c);
+            } else {
+                zero_row(sm.q[j], h);
             }
-        } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(slab + sw128(h, c)) = make_uint4(0, 0, 0, 0);
         }
+        cp_async_commit();
+        cp_async_wait_all();
+        for (int h = lane; h < H && h < kHp; h += 32) bf16_row_to_f16(sm.q[j], h);
+    }
+    const int wcount = P.win_count[b];
+    const int wlen = wcount < WIN ? (wcount < 0 ? 0 : wcount) : WIN;
+    const int n = (K > 0) ? entries_of(P.cache, b) : 0;
+    // Bring this unit's selected entries and window ring into L2 now, so that
+    // every tile's gather below is served from L2 rather than waiting on DRAM.
+    {
+        const int p_end = min(K, t_end * kT);
+        for (int pos = t_begin * kT + tid; pos < p_end; pos += kThreads) {
+            const int e = P.idx[(int64_t)b * K + pos];
+            if (e >= 0 && e < n) {
+                const int pg = page_of(P.cache, b, e);
+                if (pg >= 0) {
+                    const int64_t ent = (int64_t)pg * PAGE + (e % PAGE);
+                    bulk_prefetch_l2(P.cache.main_codes + ent * MCB, MCB);
+                    bulk_prefetch_l2(P.cache.main_scales + ent * MSB, MSB);
+                }
+            }
+        }
+        if (tid == 0 && t_end * kT > K && wlen > 0)
+            bulk_prefetch_l2(P.win + (int64_t)b * WIN * D, (uint32_t)wlen * D * 2);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
-    const int wcount = P.win_count[b];
-    const int wlen = wcount < WIN ? (wcount < 0 ? 0 : wcount) : WIN;
-    const int n = (K > 0) ? entries_of(P.cache, b) : 0;
-    uint32_t phase = 0;
+    uint32_t phase = 0, wphase = 0;
     bool o_init = false;
     bool timed_out = false;
 
     const uint32_t idesc_s = idesc_f16(128, kHp, 0, 0, 0);
     const uint32_t idesc_o = idesc_f16(128, kHp, 0, 1, 1);
+    const uint64_t desc_items = smem_desc(sm.items[0], 16, 1024, kLayoutSw128);
+    const uint64_t desc_q = smem_desc(sm.q[0], 16, 1024, kLayoutSw128);
+    const uint64_t desc_vt = smem_desc(sm.items[0], 16384, 1024, kLayoutSw128);
+    const uint64_t desc_p = smem_desc(sm.p, 16384, 1024, kLayoutSw128);
 
-    for (int t = t_begin; t < t_end && !timed_out; ++t) {
-        // ---- gather + dequantise 128 items: thread = slab j of items r0 + 32 i (i < 4).
-        // The dependent loads (index -> page -> bytes) of the four items are issued
-        // stage by stage so their latencies overlap.
-        {
-            const int j = tid & 7, r0 = tid >> 3;
-            int ent_i[4];
-            int64_t ent_row[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int pos = t * kT + r0 + 32 * i;
-                ent_i[i] = (pos < K) ? __ldg(P.idx + (int64_t)b * K + pos) : -1;
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                ent_row[i] = -1;
-                const int e = ent_i[i];
+    // Where each item of tile t comes from (one thread per item), into buffer buf.
+    auto lookup = [&](int t, int buf) {
+        if (tid < kT) {
+            const int pos = t * kT + tid;
+            int kind = 0;
+            int64_t row = -1;
+            if (pos < K) {
+                const int e = P.idx[(int64_t)b * K + pos];
                 if (e >= 0 && e < n) {
                     const int pg = page_of(P.cache, b, e);
-                    if (pg >= 0) ent_row[i] = (int64_t)pg * PAGE + (e % PAGE);
-                }
-            }
-            uint4 c0[4], c1[4];
-            uint32_t swd[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                if (ent_row[i] >= 0) {
-                    const uint4* cs = reinterpret_cast<const uint4*>(P.cache.main_codes + ent_row[i] * MCB + 32 * j);
-                    c0[i] = __ldg(cs);
-                    c1[i] = __ldg(cs + 1);
-                    swd[i] = __ldg(reinterpret_cast<const uint32_t*>(P.cache.main_scales + ent_row[i] * MSB + 4 * j));
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = r0 + 32 * i;
-                const int pos = t * kT + r;
-                uint8_t* slab = sm.items[j];
-                bool ok = false;
-                if (ent_row[i] >= 0) {
-                    ok = true;
-                    const uint32_t cw[8] = {c0[i].x, c0[i].y, c0[i].z, c0[i].w, c1[i].x, c1[i].y, c1[i].z, c1[i].w};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {  // chunk c: channels 8c..8c+7, scale byte c/2
-                        const __half2 s2 = __float2half2_rn(e4m3_decode_pos((swd[i] >> (8 * (c >> 1))) & 0xFFu));
-                        uint4 o;
-                        uint32_t* os = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const __half2 v = __hmul2(sm.lut[(cw[c] >> (8 * k)) & 0xFFu], s2);
-                            os[k] = *reinterpret_cast<const uint32_t*>(&v);
-                        }
-                        *reinterpret_cast<uint4*>(slab + sw128(r, c)) = o;
-                    }
-                } else if (pos >= K && pos - K < wlen) {
-                    ok = true;
-                    const uint4* src = reinterpret_cast<const uint4*>(P.win + ((int64_t)b * WIN + (pos - K)) * D + 64 * j);
-                    uint4 wv[8];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) wv[c] = __ldg(src + c);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t ws[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
-                        uint4 o;
-                        uint32_t* os = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const __half2 hv = __floats2half2_rn(__uint_as_float(ws[k] << 16),
-                                                                 __uint_as_float(ws[k] & 0xFFFF0000u));
-                            os[k] = *reinterpret_cast<const uint32_t*>(&hv);
-                        }
-                        *reinterpret_cast<uint4*>(slab + sw128(r, c)) = o;
+                    if (pg >= 0) {
+                        kind = 1;
+                        row = (int64_t)pg * PAGE + (e % PAGE);
                     }
                 }
-                if (!ok) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(slab + sw128(r, c)) = make_uint4(0, 0, 0, 0);
-                }
-                if (j == 0) sm.valid[r] = ok;
+            } else if (pos - K < wlen) {
+                kind = 2;
             }
+            sm.kind[buf][tid] = kind;
+            sm.src_row[buf][tid] = row;
+            const unsigned ent = __ballot_sync(0xffffffffu, kind == 1);
+            const unsigned win = __ballot_sync(0xffffffffu, kind == 2);
+            if (lane == 0) {
+                if (ent) atomicAdd(&sm.n_entries[buf], __popc(ent));
+                if (win) sm.has_window[buf] = 1;
+            }
+        }
+    };
+    // Packed bytes of the tile's cache entries: warp = slab j, lane = rows lane + 32 i.
+    uint4 raw0[4], raw1[4];
+    uint32_t raws[4];
+    auto load_entries = [&](int buf) {
+        const int j = warp;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = lane + 32 * i;
+            if (sm.kind[buf][r] == 1) {
+                const int64_t ent = sm.src_row[buf][r];
+                const uint4* cs = reinterpret_cast<const uint4*>(P.cache.main_codes + ent * MCB + 32 * j);
+                raw0[i] = __ldg(cs);
+                raw1[i] = __ldg(cs + 1);
+                raws[i] = __ldg(reinterpret_cast<const uint32_t*>(P.cache.main_scales + ent * MSB + 4 * j));
+            } else {
+                raw0[i] = raw1[i] = make_uint4(0, 0, 0, 0);
+                raws[i] = 0;
+            }
+        }
+    };
+
+    int buf = 0;
+    if (t_begin < t_end) {
+        lookup(t_begin, 0);
+        __syncthreads();
+        load_entries(0);
+    }
+    for (int t = t_begin; t < t_end && !timed_out; ++t, buf ^= 1) {
+        const bool has_window = sm.has_window[buf] != 0;
+        // ---- window rows by TMA, one 64-channel box per slab (O of the previous
+        // tile has completed, so the item buffer is free)
+        if (tid == 0 && has_window) {
+            mbar_expect_tx(&sm.wbar, 8 * kT * 128);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) tma_load_3d(sm.items[j], &maps.win[prob], 64 * j, t * kT - K, b, &sm.wbar);
+        }
+        // ---- cache entries (bytes already in registers): warp = slab, lane = row.
+        // The window boxes cover all 128 rows, so they must land first.
+        if (has_window) {
+            if (!mbar_wait(&sm.wbar, wphase)) timed_out = true;
+            wphase ^= 1;
+        }
+        {
+            const int j = warp;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = lane + 32 * i;
+                const int kind = sm.kind[buf][r];
+                if (kind == 2) {
+                    bf16_row_to_f16(sm.items[j], r);
+                } else if (kind == 0) {
+                    zero_row(sm.items[j], r);
+                } else {
+                    const uint32_t cw[8] = {raw0[i].x, raw0[i].y, raw0[i].z, raw0[i].w,
+                                            raw1[i].x, raw1[i].y, raw1[i].z, raw1[i].w};
+#pragma unroll
+                    for (int c2 = 0; c2 < 4; ++c2) {  // chunks 2*c2, 2*c2+1 share scale byte c2
+                        const __half2 s2 = __float2half2_rn(e4m3_decode_pos((raws[i] >> (8 * c2)) & 0xFFu));
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int c = 2 * c2 + cc;
+                            uint4 o;
+                            uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint32_t h = e2m1x2_to_h2((cw[c] >> (8 * k)) & 0xFFu);
+                                const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&h), s2);
+                                os[k] = *reinterpret_cast<const uint32_t*>(&v);
+                            }
+                            *reinterpret_cast<uint4*>(sm.items[j] + sw128(r, c)) = o;
+                        }
+                    }
+                }
+            }
+        }
+        if (tid == 0) {
+            sm.n_entries[buf ^ 1] = 0;
+            sm.has_window[buf ^ 1] = 0;
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(timed_out)) {
+            timed_out = true;
+            break;
+        }
 
-        // ---- S^T = Items . Q^T
+        // ---- S^T = Items . Q^T, and meanwhile the next tile's lookups
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll 1
             for (int ks = 0; ks < 32; ++ks) {  // 16 latent channels per MMA
-                const int j = ks >> 2, off = (ks & 3) * 32;
-                const uint64_t a = smem_desc(sm.items[j] + off, 16, 1024, kLayoutSw128);
-                const uint64_t bq = smem_desc(sm.q[j] + off, 16, 1024, kLayoutSw128);
-                tc_mma_f16(tbase + kColS, a, bq, idesc_s, ks > 0 ? 1u : 0u);
+                const uint32_t off = (uint32_t)((ks >> 2) * (kT * 128) + (ks & 3) * 32) >> 4;
+                const uint32_t offq = (uint32_t)((ks >> 2) * (kHp * 128) + (ks & 3) * 32) >> 4;
+                tc_mma_f16(tbase + kColS, desc_items + off, desc_q + offq, idesc_s, ks > 0 ? 1u : 0u);
             }
             tc_commit(&sm.bar);
         }
+        if (t + 1 < t_end) lookup(t + 1, buf ^ 1);
         if (!mbar_wait(&sm.bar, phase)) timed_out = true;
         phase ^= 1;
         if (__syncthreads_or(timed_out)) {
@@ -260,17 +344,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_mma(const __grid_constant_
         }
         tc_fence_after();
 
-        // ---- softmax statistics (warps 0-3: thread = item row)
-        const uint32_t s_addr = tbase + ((uint32_t)((warp & 3) * 32) << 16) + kColS;
-        if (warp < 4) {
-            float v[64];
-            tmem_ld_32x32b_x64(s_addr, v);
-            const bool ok = sm.valid[warp * 32 + lane] != 0;
+        // ---- softmax statistics: warp = (quadrant, head half); thread = item row
+        const int quad = warp & 3, hh = warp >> 2;
+        const int row = quad * 32 + lane;
+        const uint32_t s_addr = tbase + ((uint32_t)(quad * 32) << 16) + kColS + 32 * hh;
+        const bool ok = sm.kind[buf][row] != 0;
+        {
+            float v[32];
+            tmem_ld_32x32b_x32(s_addr, v);
 #pragma unroll
-            for (int h = 0; h < 64; ++h) v[h] = ok ? v[h] * ab.scale : -INFINITY;
-            warp_reduce_scatter64<true>(v);
-            sm.red[warp][2 * lane] = v[0];
-            sm.red[warp][2 * lane + 1] = v[1];
+            for (int h = 0; h < 32; ++h) v[h] = ok ? v[h] * ab.scale : -INFINITY;
+            warp_reduce_scatter<true, 32>(v);
+            sm.red[quad][32 * hh + lane] = v[0];
         }
         __syncthreads();
         bool rescale = false;
@@ -288,36 +373,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_mma(const __grid_constant_
         rescale = __syncthreads_or(rescale);
 
         // ---- P^T = exp(s - m) in fp16 (S reloaded from TMEM), row sums of the rounded p
-        if (warp < 4) {
-            const int r = warp * 32 + lane;
-            float v[64];
-            tmem_ld_32x32b_x64(s_addr, v);
-            const bool ok = sm.valid[r] != 0;
+        {
+            float v[32];
+            tmem_ld_32x32b_x32(s_addr, v);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 uint4 o;
                 uint32_t* os = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int h = 8 * c + 2 * k;
-                    const float p0 = ok ? __expf(v[h] * ab.scale - sm.m_used[h]) : 0.0f;
-                    const float p1 = ok ? __expf(v[h + 1] * ab.scale - sm.m_used[h + 1]) : 0.0f;
+                    const float p0 = ok ? __expf(v[h] * ab.scale - sm.m_used[32 * hh + h]) : 0.0f;
+                    const float p1 = ok ? __expf(v[h + 1] * ab.scale - sm.m_used[32 * hh + h + 1]) : 0.0f;
                     const __half2 hv = __floats2half2_rn(p0, p1);
                     const float2 back = __half22float2(hv);
                     v[h] = back.x;
                     v[h + 1] = back.y;
                     os[k] = *reinterpret_cast<const uint32_t*>(&hv);
                 }
-                *reinterpret_cast<uint4*>(sm.p + sw128(r, c)) = o;
+                *reinterpret_cast<uint4*>(sm.p + sw128(row, 4 * hh + c)) = o;
             }
-            warp_reduce_scatter64<false>(v);
-            sm.red[warp][2 * lane] = v[0];
-            sm.red[warp][2 * lane + 1] = v[1];
+            warp_reduce_scatter<false, 32>(v);
+            // the max pass read red[] before the barrier above; reuse it for sums
+            sm.red[quad][32 * hh + lane] = v[0];
         }
         // ---- rescale O^T where a head's reference maximum moved
         if (rescale) {
-            const int quad = warp & 3;
-            for (int c = (warp >> 2) * 2; c < (warp >> 2) * 2 + 2; ++c) {
+            for (int c = hh * 2; c < hh * 2 + 2; ++c) {
                 const uint32_t ta = tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * c;
                 float o[64];
                 tmem_ld_32x32b_x64(ta, o);
@@ -339,14 +421,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_mma(const __grid_constant_
             for (int c = 0; c < 4; ++c) {
 #pragma unroll 1
                 for (int i = 0; i < 8; ++i) {  // 16 items per MMA
-                    const uint64_t a = smem_desc(sm.items[2 * c] + 2048 * i, 16384, 1024, kLayoutSw128);
-                    const uint64_t bp = smem_desc(sm.p + 2048 * i, 16384, 1024, kLayoutSw128);
-                    tc_mma_f16(tbase + kColO + 64 * c, a, bp, idesc_o, (o_init || i > 0) ? 1u : 0u);
+                    const uint32_t offa = (uint32_t)(2 * c * (kT * 128) + 2048 * i) >> 4;
+                    const uint32_t offp = (uint32_t)(2048 * i) >> 4;
+                    tc_mma_f16(tbase + kColO + 64 * c, desc_vt + offa, desc_p + offp, idesc_o,
+                               (o_init || i > 0) ? 1u : 0u);
                 }
             }
             tc_commit(&sm.bar);
         }
         o_init = true;
+        if (t + 1 < t_end) load_entries(buf ^ 1);  // in flight while O runs
         if (!mbar_wait(&sm.bar, phase)) timed_out = true;
         phase ^= 1;
         if (__syncthreads_or(timed_out)) {
@@ -384,6 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_mma(const __grid_constant_
             ab.part_ml[((int64_t)unit * H + tid) * 2 + 0] = sm.m_used[tid];
             ab.part_ml[((int64_t)unit * H + tid) * 2 + 1] = sm.l[tid];
         }
+    }
+    // a timed-out wait may leave copies in flight: let them land before the CTA exits
+    if (tid == 0) {
+        (void)mbar_wait(&sm.wbar, wphase ^ 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -452,8 +540,41 @@ size_t attn_mma_workspace_bytes(int n_problems, int batch, int H, int Kmax) {
     return units * H * D * sizeof(float) + units * H * 2 * sizeof(float);
 }
 
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 attn_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// Window ring [batch][128][512] bf16 as a 3-D tensor, boxes of 64 channels x 128 rows.
+bool make_window_map(CUtensorMap* m, const void* base, int batch) {
+    auto fn = attn_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)WIN, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)WIN * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)WIN, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_attn_mma(const AttnBatch& ab_in, cudaStream_t st, cudaEvent_t* ev) {
     AttnBatch ab = ab_in;
+    AttnMaps maps;  // kernel parameter (copied at launch)
+    std::memset(&maps, 0, sizeof(maps));
+    for (int i = 0; i < ab.n; ++i)
+        if (!make_window_map(&maps.win[i], ab.p[i].win, ab.batch)) return cudaErrorInvalidValue;
     const int splits = attn_mma_splits(ab.n, ab.batch, ab.Kmax);
     const int tiles = (ab.Kmax + WIN + kT - 1) / kT;
     const int tps = (tiles + splits - 1) / splits;
@@ -467,7 +588,7 @@ cudaError_t launch_attn_mma(const AttnBatch& ab_in, cudaStream_t st, cudaEvent_t
         return true;
     }();
     (void)attr;
-    k_attn_mma<<<ab.n * ab.batch * splits, kThreads, smem, st>>>(ab, splits, tps);
+    k_attn_mma<<<ab.n * ab.batch * splits, kThreads, smem, st>>>(ab, maps, splits, tps);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (ev) cudaEventRecord(ev[0], st);

@@ -11,7 +11,7 @@
 // two MMAs of K = 64 each; the epilogue applies ReLU, the head weights and the
 // head sum, one thread per entry row.
 //
-// Persistent, warp-specialised CTA (192 threads, two CTAs per SM):
+// Persistent, warp-specialised CTA (320 threads, two CTAs per SM):
 //   warp 0  producer: TMA tile loads of the keys (one 64-entry page per box,
 //           64-byte swizzle) and bulk copies of their E8M0 scales into an
 //           8-stage ring; per work item also the query tile, its scales and
@@ -19,8 +19,9 @@
 //   warp 1  MMA issuer: rearranges each stage's scales into the 32x128-bit
 //           layout tcgen05.cp copies into TMEM, then issues the two MMAs into
 //           one of two TMEM accumulators and commits the stage back.
-//   warps 2-5 epilogue: one TMEM lane (= entry) per thread: tcgen05.ld of the
-//           64 head columns, ReLU, weight, sum, one fp32 score store.
+//   warps 2-9 epilogue, two groups of four (one TMEM lane quadrant per warp);
+//           group g drains accumulator g (every other tile): tcgen05.ld of the
+//           64 head columns of its entry, ReLU, weight, sum, one score store.
 // Work item = (problem, sequence, chunk of kChunkTiles tiles), round-robin over
 // the grid.  Every wait is bounded; a timeout sets CSA2_DEVERR_TIMEOUT in the
 // problem's status word and the CTA drains and exits.
@@ -44,7 +45,7 @@ constexpr int kHeads = 64;        // MMA N (indexer heads)
 constexpr int kStages = 8;
 constexpr int kTile = 128;        // entries per MMA tile (MMA M)
 constexpr int kChunkTiles = 16;   // tiles per work item
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;     // producer, MMA issuer, 2 x 4 epilogue warps
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColAcc = 0;         // 2 x 64 accumulator columns
 constexpr uint32_t kColSfa = 128;       // kStages x 4 scale columns (A)
@@ -73,6 +74,8 @@ struct __align__(1024) Smem {
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory beyond the 227 KB per-block limit");
+
 
 struct Item {
     int p, b, t0, t1, n;
@@ -116,9 +119,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.bfull[i], 1);
-            mbar_init(&sm.bempty[i], 1 + 4);
+            mbar_init(&sm.bempty[i], 1 + 8);
             mbar_init(&sm.tfull[i], 1);
-            mbar_init(&sm.tempty[i], 4);
+            mbar_init(&sm.tempty[i], 4);  // the four warps of epilogue group i
         }
         mbar_init(&sm.drained, 1);
         sm.abort = 0;
@@ -271,9 +274,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
+        // Group g = (warp - 2) / 4 drains accumulator g, i.e. every other tile.
+        const int grp = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
-        uint32_t bslot = 0, bphase = 0, acc = 0, aphase = 0;
+        uint32_t bslot = 0, bphase = 0, aphase = 0, tile_no = 0;
         for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
             Item it;
             if (!item_at(sb, mp, id, it)) continue;
@@ -282,14 +287,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float* w = sm.w[bslot];
             float* out = P.scores + (int64_t)it.b * sb.score_stride;
             bool stop = false;
-            for (int t = it.t0; t < it.t1; ++t) {
-                if (!mbar_wait_warp(&sm.tfull[acc], aphase)) { raise_abort(sm, P.cache.status); stop = true; break; }
+            for (int t = it.t0; t < it.t1; ++t, ++tile_no) {
+                if ((int)(tile_no & 1u) != grp) continue;
+                if (!mbar_wait_warp(&sm.tfull[grp], aphase)) { raise_abort(sm, P.cache.status); stop = true; break; }
+                aphase ^= 1;
                 tc_fence_after();
                 float v[64];
-                tmem_ld_32x32b_x64(tbase + ((uint32_t)(quad * 32) << 16) + kColAcc + kHeads * acc, v);
+                tmem_ld_32x32b_x64(tbase + ((uint32_t)(quad * 32) << 16) + kColAcc + kHeads * grp, v);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.tempty[acc]);
+                if (lane == 0) mbar_arrive(&sm.tempty[grp]);
                 float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent chains
 #pragma unroll
                 for (int h = 0; h < kHeads; h += 4) {
@@ -302,8 +309,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float s = (part[0] + part[1]) + (part[2] + part[3]);
                 const int e = t * kTile + row;
                 if (e < it.n) out[e] = s;
-                acc ^= 1;
-                if (acc == 0) aphase ^= 1;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.bempty[bslot]);

@@ -26,6 +26,7 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kSamples = 2048;
 constexpr int kCap = 12288;
+constexpr int kRun = 16;  // contiguous scores per thread per pass
 
 struct TopkSmem {
     uint32_t key[kCap];
@@ -35,6 +36,8 @@ struct TopkSmem {
     int sel[2];
     int flag;
 };
+static_assert(sizeof(TopkSmem) + 1024 <= 232448, "shared memory beyond the 227 KB per-block limit");
+
 
 // Exclusive prefix sum of one int per thread over the block; returns the total.
 __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* excl) {
@@ -112,28 +115,48 @@ __device__ void radix_select(KeyAt key_at, int cnt, int k, TopkSmem& sm, uint32_
 }
 
 // Ordered compaction of the Top-K: keys above kth, then (in index order) the
-// first `need` keys equal to it.  Writes out positions [0, K).
+// first `need` keys equal to it.  Writes out positions [0, K).  Each thread
+// takes a contiguous run of kRun keys per round.
 template <class KeyAt, class IdxAt>
 __device__ void emit_topk(KeyAt key_at, IdxAt idx_at, int cnt, uint32_t kth, int need, int K,
                           TopkSmem& sm, int32_t* io, float* so) {
-    int base = 0, eq_seen = 0;
-    for (int i0 = 0; i0 < cnt; i0 += kThreads) {
-        const int i = i0 + threadIdx.x;
-        const uint32_t kk = i < cnt ? key_at(i) : 0u;
-        const int gt = (i < cnt) && (kk > kth);
-        const int eq = (i < cnt) && (kk == kth);
+    int base_out = 0, eq_seen = 0;
+    for (int base = 0; base < cnt; base += kThreads * kRun) {
+        const int i0 = base + threadIdx.x * kRun;
+        uint32_t kk[kRun];
+        int gt = 0, eq = 0;
+#pragma unroll
+        for (int v = 0; v < kRun; ++v) {
+            kk[v] = (i0 + v < cnt) ? key_at(i0 + v) : 0u;
+            gt += (i0 + v < cnt) && (kk[v] > kth);
+            eq += (i0 + v < cnt) && (kk[v] == kth);
+        }
         int eq_rank;
         const int eq_tot = block_excl_scan(eq, sm.warp_tot, &eq_rank);
-        const int take = gt || (eq && (eq_seen + eq_rank) < need);
+        // equal keys this thread may take: those whose rank among equals is < need
+        const int eq_take = max(0, min(eq, need - (eq_seen + eq_rank)));
         int pos;
-        const int take_tot = block_excl_scan(take, sm.warp_tot, &pos);
-        if (take && base + pos < K) {
-            io[base + pos] = idx_at(i);
-            if (so) so[base + pos] = order_key_f32(kk);
+        const int take_tot = block_excl_scan(gt + eq_take, sm.warp_tot, &pos);
+        int o = base_out + pos, e_left = eq_take;
+#pragma unroll
+        for (int v = 0; v < kRun; ++v) {
+            if (i0 + v >= cnt) continue;
+            bool take = kk[v] > kth;
+            if (kk[v] == kth && e_left > 0) {
+                take = true;
+                --e_left;
+            }
+            if (take) {
+                if (o < K) {
+                    io[o] = idx_at(i0 + v);
+                    if (so) so[o] = order_key_f32(kk[v]);
+                }
+                ++o;
+            }
         }
-        base += take_tot;
+        base_out += take_tot;
         eq_seen += eq_tot;
-        if (base >= K) break;
+        if (base_out >= K) break;
     }
 }
 
@@ -168,18 +191,41 @@ __global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanB
         radix_select([&](int i) { return sm.key[i]; }, kSamples, rank, sm, &guess, &unused);
     }
 
-    // 2. one pass: ordered compaction of the scores at or above the guess
+    // 2. one pass: ordered compaction of the scores at or above the guess.  Each
+    // thread takes a contiguous run of kRun scores, so a chunk of kThreads * kRun
+    // scores costs four vector loads and one block scan per thread.
     int cnt = 0;
     bool fits = true;
-    for (int i0 = 0; i0 < n; i0 += kThreads) {
-        const int i = i0 + tid;
-        const uint32_t kk = i < n ? f32_order_key(row[i]) : 0u;
-        const int c = (i < n) && (kk >= guess);
+    for (int base = 0; base < n; base += kThreads * kRun) {
+        const int i0 = base + tid * kRun;
+        uint32_t kk[kRun];
+        if (i0 + kRun <= n) {
+#pragma unroll
+            for (int v = 0; v < kRun / 4; ++v) {
+                const float4 f = *reinterpret_cast<const float4*>(row + i0 + 4 * v);
+                kk[4 * v] = f32_order_key(f.x);
+                kk[4 * v + 1] = f32_order_key(f.y);
+                kk[4 * v + 2] = f32_order_key(f.z);
+                kk[4 * v + 3] = f32_order_key(f.w);
+            }
+        } else {
+#pragma unroll
+            for (int v = 0; v < kRun; ++v) kk[v] = (i0 + v < n) ? f32_order_key(row[i0 + v]) : 0u;
+        }
+        int c = 0;
+#pragma unroll
+        for (int v = 0; v < kRun; ++v) c += (i0 + v < n) && (kk[v] >= guess);
         int pos;
         const int tot = block_excl_scan(c, sm.warp_tot, &pos);
-        if (c && cnt + pos < kCap) {
-            sm.key[cnt + pos] = kk;
-            sm.idx[cnt + pos] = i;
+        if (cnt + tot <= kCap) {
+            int o = cnt + pos;
+#pragma unroll
+            for (int v = 0; v < kRun; ++v)
+                if ((i0 + v < n) && (kk[v] >= guess)) {
+                    sm.key[o] = kk[v];
+                    sm.idx[o] = i0 + v;
+                    ++o;
+                }
         }
         cnt += tot;
         if (cnt > kCap) {

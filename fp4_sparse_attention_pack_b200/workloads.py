@@ -139,6 +139,8 @@ WORKLOADS = {
 PROFILE_WORKLOADS = {
     # one Full layer over 32 sequences x 65,536 entries: 142 MB of indexer keys per scan
     "scan32": Workload("scan32_1layer_b32_128k", 5, 32, 131072, single_full(), 64, 64, 512, 4),
+    # the 40-layer step at batch 4: 160 attention units (about one wave), 410 MB of keys per step
+    "step_b4": Workload("step_b4_40layer_128k", 6, 4, 131072, schedule_alternating_40(), 64, 64, 512, 4),
 }
 
 
