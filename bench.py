@@ -119,42 +119,60 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-def scan_traffic(kernel_file: str):
-    """Per-launch DRAM bytes of the scan from a committed ncu summary, only while
-    the kernel source is unchanged since the capture (else None)."""
-    p = os.path.join(ROOT, "profiles", "scan_traffic.json")
+KERNEL_SOURCES = {"index_scan": "scan_mma.cu", "attention": "attn_mma.cu", "topk": "topk.cu"}
+
+
+def kernel_traffic(kernel: str):
+    """Per-launch DRAM bytes (read + write) of a kernel at the bench workload from
+    the committed ncu summary profiles/<kernel>_traffic.json, only while the
+    kernel's source is unchanged since the capture (else None)."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")
+    src = os.path.join(ROOT, "fp4_sparse_attention_pack_b200", "csrc", KERNEL_SOURCES[kernel])
     try:
         with open(p) as f:
             d = json.load(f)
-        with open(kernel_file, "rb") as f:
+        with open(src, "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()[:16]
-        if d.get("source_sha") != sha:
-            return None, d
-        return d, d
+        return d.get("bytes_per_launch_at_workload") if d.get("source_sha") == sha else None
     except (OSError, ValueError):
-        return None, None
+        return None
 
 
-def step_bytes(wl, n_entries):
-    """Algorithmic HBM bytes of one decode step (our accounting of the path):
-    every scan reads its source's keys (68 B/entry) and its query; every
-    attention reads K entries (288 B) + indices and the 128-token window and
-    its query; outputs fp32; the cache write of the completed groups."""
+def workload_config(wl, world):
+    """The workload keys of the JSON line's config (both arms)."""
+    return {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.T,
+            "layers": wl.table.n_layers, "scans_per_step": len(wl.table.scan_layers()), "H": wl.H,
+            "H_idx": wl.H_idx, "top_k": wl.K, "parallelism": f"dp{world} (replicas, no collective)",
+            "cache_format": "E2M1+E4M3/16 main, MXFP4 indexer keys"}
+
+
+def kernel_bytes(wl, n_entries):
+    """Algorithmic HBM bytes per launch of each kernel in one decode step (our
+    accounting of the path; every launch covers all layers of the step):
+      index_scan  each scanned source's indexer keys once (64 code + 4 scale
+                  bytes per entry), every scan's query (64 x (64 + 4) bytes) and
+                  head weights, one fp32 score per (scan, entry) written;
+      topk        the scores read, K indices written per (scan, sequence);
+      attention   per (layer, sequence) the K selected entries (256 code + 32
+                  scale bytes) and their indices, the 128-token bf16 window, the
+                  bf16 query, the fp32 output;
+      step        all kernels, plus the cache write of the new tokens."""
     t = wl.table
     B, H, Hi, K = wl.B, wl.H, wl.H_idx, wl.K
-    rd = wr = 0
-    scan_rd = 0
-    for l in t.scan_layers():
-        n = sum(n_entries[t.src[l]])
-        scan_rd += n * 68 + B * (Hi * 128 * 2 + Hi * 4)
-        wr += B * K * 4
-    rd += scan_rd
-    for l, m in enumerate(t.mode):
-        rd += B * (WIN * 512 * 2 + H * 512 * 2)
+    scans = t.scan_layers()
+    n_src = {s: sum(n_entries[s]) for s in range(t.n_sources)}
+    scanned = sorted({t.src[l] for l in scans})
+    score_bytes = sum(n_src[t.src[l]] * 4 for l in scans)
+    scan = (sum(n_src[s] * 68 for s in scanned) + len(scans) * B * Hi * (64 + 4 + 4) + score_bytes)
+    topk = score_bytes + len(scans) * B * K * 4
+    attn = 0
+    for m in t.mode:
+        attn += B * (WIN * 512 * 2 + H * 512 * 2 + H * 512 * 4)
         if m != 0:
-            rd += B * K * (288 + 4)
-        wr += B * H * 512 * 4
-    return rd, wr, scan_rd
+            attn += B * K * (288 + 4)
+    cache_write = t.n_sources * B * (512 * 2 + 4 + 288 + 68)
+    return {"index_scan": scan, "topk": topk, "attention": attn,
+            "step": scan + topk + attn + cache_write + t.n_layers * B * 1024}
 
 
 WIN = 128
@@ -261,7 +279,7 @@ def run_reference(args, rank):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.T, "layers": t.n_layers},
+            "config": workload_config(wl, 1),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
                              "sample": desc},
@@ -395,35 +413,37 @@ def run_ours(args, rank, world, local_rank):
 
     L = wl.table.n_layers
     value = L * world / (ms / 1e3)
-    rd, wr, scan_rd = step_bytes(wl, n_ent)
+    kb = kernel_bytes(wl, n_ent)
     peak, peak_kind = measured_peaks()
-    scan_ms = phase_ms["index_scan"]
-    achieved = scan_rd / (scan_ms / 1e3) / 1e9
-    tr, _ = scan_traffic(os.path.join(ROOT, "fp4_sparse_attention_pack_b200", "csrc", "scan.cu"))
-    traffic = tr["bytes_per_launch_at_workload"] if tr else None
-    launches_per_step = 1 + 2 * dm.S + 3 + 2
+    # roofline of the kernel with the largest share of the step
+    dom = max(("index_scan", "attention", "topk"), key=lambda k: phase_ms[k])
+    kernels = {k: {"algorithmic_bytes_per_launch": kb[k], "launch_ms": phase_ms[k],
+                   "achieved_gbs": kb[k] / (phase_ms[k] / 1e3) / 1e9,
+                   "frac_of_measured_hbm": kb[k] / (phase_ms[k] / 1e3) / 1e9 / peak,
+                   "dram_bytes_per_launch": kernel_traffic(k)}
+               for k in ("index_scan", "topk", "attention")}
+    achieved = kernels[dom]["achieved_gbs"]
+    launches_per_step = csa.layer_step_launches(dm.model, dm._in)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
-        "config": {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.T,
-                   "layers": L, "scans_per_step": len(wl.table.scan_layers()), "H": wl.H,
-                   "H_idx": wl.H_idx, "top_k": wl.K, "parallelism": f"dp{world} (replicas, no collective)",
-                   "cache_format": "E2M1+E4M3/16 main, MXFP4 indexer keys",
-                   "l2": "inputs larger than L2: %.2f GB read per step" % (rd / 1e9),
-                   "cuda_graph": True},
-        "hbm": {"step_read_bytes": rd, "step_write_bytes": wr,
-                "achieved_gbs": (rd + wr) / (ms / 1e3) / 1e9,
-                "frac_of_8tbs": (rd + wr) / (ms / 1e3) / 8e12,
-                "frac_of_measured": (rd + wr) / (ms / 1e3) / (peak * 1e9)},
-        "roofline": {"kernel": "index_scan", "bound": "hbm", "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": peak_kind, "algorithmic_bytes_per_launch": scan_rd,
-                     "launch_ms": scan_ms},
+        "config": dict(workload_config(wl, world),
+                       l2="inputs larger than L2: %.2f GB read per step" % (kb["step"] / 1e9),
+                       cuda_graph=True),
+        "hbm": {"step_algorithmic_bytes": kb["step"],
+                "achieved_gbs": kb["step"] / (ms / 1e3) / 1e9,
+                "frac_of_measured": kb["step"] / (ms / 1e3) / (peak * 1e9)},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": kernels[dom]["dram_bytes_per_launch"],
+                     "peak_source": peak_kind, "algorithmic_bytes_per_launch": kb[dom],
+                     "launch_ms": phase_ms[dom]},
+        "kernels": kernels,
         "phase_ms": phase_ms,
         "e2e": {"value": L * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches_per_step": launches_per_step,
         "clocks": clocks.summary(t_wall0, t_wall1),
         "device_status": status,
     }

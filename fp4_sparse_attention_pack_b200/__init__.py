@@ -14,7 +14,7 @@ from ._build import LIB
 
 __all__ = ["Csa2Error", "lib", "csa2_cache", "csa2_window", "csa2_model", "csa2_step_in",
            "csa2_step_out", "pack_cache", "index_topk", "index_topk_workspace", "sparse_attn",
-           "sparse_attn_workspace", "window_append", "layer_step", "layer_step_workspace",
+           "sparse_attn_workspace", "window_append", "layer_step", "layer_step_workspace", "layer_step_launches",
            "SWA_ONLY", "FULL", "REINDEX", "REUSE", "DTYPE_BF16", "DTYPE_F32"]
 
 SWA_ONLY, FULL, REINDEX, REUSE = 0, 1, 2, 3
@@ -84,6 +84,7 @@ def lib():
             ("csa2_layer_step_workspace", _sz, [P(csa2_model)]),
             ("csa2_layer_step", ctypes.c_int, [P(csa2_model), P(csa2_step_in), P(csa2_step_out), _vp,
                                                _sz, _vp]),
+            ("csa2_layer_step_launches", ctypes.c_int, [P(csa2_model), P(csa2_step_in)]),
         ]:
             f = getattr(L, name)
             f.restype = res
@@ -151,6 +152,14 @@ def layer_step(model: csa2_model, step_in: csa2_step_in, step_out: csa2_step_out
     _ok(lib().csa2_layer_step(ctypes.byref(model), ctypes.byref(step_in), ctypes.byref(step_out),
                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
         "csa2_layer_step")
+
+
+def layer_step_launches(model: csa2_model, step_in: csa2_step_in) -> int:
+    """Kernel launches one layer_step call enqueues (no work is enqueued)."""
+    n = int(lib().csa2_layer_step_launches(ctypes.byref(model), ctypes.byref(step_in)))
+    if n < 0:
+        raise Csa2Error(n, "csa2_layer_step_launches")
+    return n
 
 
 def index_topk_noalloc(cache: csa2_cache, q_idx, w, K: int, idx_out, score_out=None, stream=None):

@@ -247,6 +247,25 @@ size_t csa2_layer_step_workspace(const csa2_model* m) {
 
 namespace {
 
+// The attention batch of one step (shapes and caches; pointers filled by the caller).
+void model_attn_batch(const csa2_model* m, AttnBatch& ab) {
+    std::memset(&ab, 0, sizeof(ab));
+    ab.n = m->n_layers;
+    ab.batch = m->batch;
+    ab.H = m->H;
+    ab.Kmax = m->K;
+    ab.scale = m->scale;
+    for (int l = 0; l < m->n_layers; ++l) {
+        AttnProblem& P = ab.p[l];
+        if (m->mode[l] == CSA2_MODE_SWA_ONLY) {
+            P.K = 0;
+        } else {
+            P.K = m->K;
+            P.cache = view_of(m->caches[m->src[l]]);
+        }
+    }
+}
+
 int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step_out* out, void* ws,
                     size_t ws_bytes, csa2_stream stream, cudaEvent_t* ev) {
     int rc = check_model(m);
@@ -333,30 +352,17 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
 
     // (4) every layer attends; Reuse layers read the indices of idx_src
     AttnBatch ab;
-    std::memset(&ab, 0, sizeof(ab));
-    ab.n = L;
-    ab.batch = B;
-    ab.H = m->H;
-    ab.Kmax = m->K;
-    ab.scale = m->scale;
+    model_attn_batch(m, ab);
     const size_t units = attn_workspace_bytes(L, B, m->H, m->K) / ((D + 2) * sizeof(float));
     ab.part_o = reinterpret_cast<float*>(wsp);
     ab.part_ml = ab.part_o + units * D;
     for (int l = 0; l < L; ++l) {
         AttnProblem& P = ab.p[l];
-        const int md = m->mode[l];
         P.q = in->q[l];
         P.win = m->windows[l].tokens;
         P.win_count = m->windows[l].count;
         P.out = out->out[l];
-        if (md == CSA2_MODE_SWA_ONLY) {
-            P.K = 0;
-            P.idx = nullptr;
-        } else {
-            P.K = m->K;
-            P.cache = view_of(m->caches[m->src[l]]);
-            P.idx = out->idx[m->idx_src[l]];
-        }
+        P.idx = m->mode[l] == CSA2_MODE_SWA_ONLY ? nullptr : out->idx[m->idx_src[l]];
     }
     return cuda_status(launch_sparse_attn(ab, st, ev ? ev + 6 : nullptr));
 }
@@ -377,6 +383,22 @@ int csa2_layer_step_profiled(const csa2_model* m, const csa2_step_in* in, const 
         ev[i] = (cudaEvent_t)events[i];
     }
     return layer_step_impl(m, in, out, ws, ws_bytes, stream, ev);
+}
+
+int csa2_layer_step_launches(const csa2_model* m, const csa2_step_in* in) {
+    const int rc = check_model(m);
+    if (rc) return rc;
+    if (!in || !in->x_new) return CSA2_ERR_INVALID_ARG;
+    int n = 1;  // window append
+    for (int s = 0; s < m->n_sources; ++s)
+        if (in->x_new[s]) {
+            n += 2;  // cache write: entries, then the pending slots
+            break;
+        }
+    if (n_scans(m) > 0) n += 3;  // query quantisation, scan, Top-K
+    AttnBatch ab;
+    model_attn_batch(m, ab);
+    return n + sparse_attn_launches(ab);
 }
 
 }  // extern "C"

@@ -215,6 +215,13 @@ cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t
     return launch_attn_cuda(ab, st, ev);
 }
 
+int attn_mma_splits(int n_problems, int batch, int Kmax);
+
+int sparse_attn_launches(const AttnBatch& ab) {
+    if (attn_mma_supported(ab)) return attn_mma_splits(ab.n, ab.batch, ab.Kmax) > 1 ? 2 : 1;
+    return 2;
+}
+
 cudaError_t launch_window_append(const WinAppend& wa, cudaStream_t st) {
     dim3 grid(wa.batch, wa.n);
     k_window_append<<<grid, 64, 0, st>>>(wa);

@@ -71,6 +71,8 @@ struct AttnBatch {
 
 size_t attn_workspace_bytes(int n_problems, int batch, int H, int Kmax);
 // ev (nullable): events recorded after the split kernel and after the combine.
+// Kernel launches one launch_sparse_attn(ab) call makes.
+int sparse_attn_launches(const AttnBatch& ab);
 cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev = nullptr);
 
 // ---- window

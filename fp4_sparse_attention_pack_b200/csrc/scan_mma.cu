@@ -5,26 +5,37 @@
 //   score[b][e] = sum_h w[b][h] * max(0, qhat[b][h] . khat[b][e])
 //
 // With 64 indexer heads every key meets 64 x 128 MXFP4 products: a dense
-// contraction (about 240 flop per key byte) that CUDA cores cannot keep up
-// with at HBM speed, while the FP4 tensor cores need well under half the HBM
-// time.  Per 128-entry tile: D[128 entries x 64 heads] = K[128 x 128] . Q^T,
-// two MMAs of K = 64 each; the epilogue applies ReLU, the head weights and the
-// head sum, one thread per entry row.
+// contraction that CUDA cores cannot keep up with at HBM speed.  Several scan
+// problems (the Full and Reindex layers of one source) read the same keys, so
+// the kernel groups them: a work item is (subset of up to kMaxSub problems
+// over one cache, sequence, chunk of tiles), and each 128-entry key tile is
+// loaded once and multiplied by the queries of every problem of the subset,
+// two problems (128 query rows) per MMA pass:
+//   D[128 entries x 128 rows] = K[128 x 128] . [Q_a; Q_b]^T
+// (two MMAs of K = 64 each).  The epilogue applies ReLU, the head weights and
+// the head sum, one thread per (entry row, problem).
 //
-// Persistent, warp-specialised CTA (320 threads, two CTAs per SM):
+// Persistent, warp-specialised CTA (608 threads, one CTA per SM):
 //   warp 0  producer: TMA tile loads of the keys (one 64-entry page per box,
 //           64-byte swizzle) and bulk copies of their E8M0 scales into an
-//           8-stage ring; per work item also the query tile, its scales and
-//           the head weights.  Keys stream with an L2 evict-first policy.
-//   warp 1  MMA issuer: rearranges each stage's scales into the 32x128-bit
-//           layout tcgen05.cp copies into TMEM, then issues the two MMAs into
-//           one of two TMEM accumulators and commits the stage back.
-//   warps 2-9 epilogue, two groups of four (one TMEM lane quadrant per warp);
-//           group g drains accumulator g (every other tile): tcgen05.ld of the
-//           64 head columns of its entry, ReLU, weight, sum, one score store.
-// Work item = (problem, sequence, chunk of kChunkTiles tiles), round-robin over
-// the grid.  Every wait is bounded; a timeout sets CSA2_DEVERR_TIMEOUT in the
-// problem's status word and the CTA drains and exits.
+//           8-stage ring; per work item the query tiles, scales and head
+//           weights of every problem of the subset (double-buffered).  Keys
+//           stream with an L2 evict-first policy.
+//   warp 1  MMA issuer: copies each item's query scales and each stage's key
+//           scales into TMEM (tcgen05.cp), then per tile issues one MMA pass per
+//           problem pair into one of two TMEM accumulators, committing each pass
+//           to its epilogue group and the stage back to the producer after the
+//           last pass.
+//   warps 2-17 epilogue, two groups of eight; group g drains the passes that
+//           landed in accumulator g.  Warp w of a group reads TMEM lane quadrant
+//           w % 4 and problem (w / 4) % 2 of the pass: tcgen05.ld of the 64 head
+//           columns of its entry, ReLU, weight, sum, one score store.
+//   warp 18 scale warp: rearranges the E8M0 scales that landed in shared memory
+//           into the 32x128-bit layout tcgen05.cp reads (per item for the
+//           queries, per stage for the keys) and signals them ready, keeping
+//           the transposition and its proxy fence off the MMA issuer's path.
+// Every wait is bounded; a timeout sets CSA2_DEVERR_TIMEOUT in the problem's
+// status word and the CTA drains and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -41,35 +52,54 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kHeads = 64;        // MMA N (indexer heads)
+constexpr int kHeads = 64;        // query rows per problem
+constexpr int kPass = 2;          // problems per MMA pass (N = 128)
+constexpr int kMaxSub = 12;       // problems per work item
+constexpr int kMaxPasses = kMaxSub / kPass;
 constexpr int kStages = 8;
 constexpr int kTile = 128;        // entries per MMA tile (MMA M)
-constexpr int kChunkTiles = 16;   // tiles per work item
-constexpr int kThreads = 320;     // producer, MMA issuer, 2 x 4 epilogue warps
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColAcc = 0;         // 2 x 64 accumulator columns
-constexpr uint32_t kColSfa = 128;       // kStages x 4 scale columns (A)
-constexpr uint32_t kColSfb = 128 + 4 * kStages;  // 2 x 4 scale columns (B)
+constexpr int kMaxChunk = 16;     // tiles per work item at most (32 pages: one per producer lane)
+constexpr int kGroups = 2;        // accumulators = epilogue groups
+constexpr int kEpiWarps = 8 * kGroups;
+constexpr int kSfWarp = 2 + kEpiWarps;
+constexpr int kThreads = 32 * (kSfWarp + 1);
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColAcc = 0;                            // kGroups x 128 accumulator columns
+constexpr uint32_t kColSfa = 128 * kGroups;                // kStages x 4 scale columns (keys)
+constexpr uint32_t kColSfb = kColSfa + 4 * kStages;        // 2 x kMaxPasses x 4 (queries)
+static_assert(kColSfb + 2 * kMaxPasses * 4 <= kTmemCols, "TMEM columns");
 constexpr int kMaxSources = CSA2_MAX_SOURCES;
+
+// Problems that read one cache, scanned together.
+struct ScanSub {
+    int src;      // keys[] map index
+    int n;        // problems
+    int chunk;    // tiles per work item
+    int chunks;   // work items per sequence
+    int item0;    // first work item
+    int8_t prob[kMaxSub];
+};
 
 struct MmaScanMaps {
     CUtensorMap keys[kMaxSources];  // per distinct cache: idx codes [num_pages*64][64 B]
     CUtensorMap queries;            // [n * batch * 64][64 B]
-    int src_of[kMaxProblems];       // problem -> keys[] index
-    int chunks;                     // work items per (problem, sequence)
+    ScanSub sub[kMaxProblems];
+    int n_sub;
+    int n_items;
 };
 
 struct __align__(1024) Smem {
-    uint8_t a[kStages][kTile * 64];     // key codes, 64B-swizzled rows
-    uint8_t b[2][kHeads * 64];          // query codes, 64B-swizzled rows
+    uint8_t a[kStages][kTile * 64];          // key codes, 64B-swizzled rows
+    uint8_t b[2][kMaxSub * kHeads * 64];     // query codes of the subset, 64B-swizzled rows
     uint8_t sfa_raw[kStages][kTile * 4];
-    uint8_t sfa_tc[kStages][512];       // 32 rows x 16 B for tcgen05.cp
-    uint8_t sfb_raw[2][kHeads * 4];
-    uint8_t sfb_tc[2][512];
-    float w[2][kHeads];
-    uint64_t full[kStages], empty[kStages];
-    uint64_t bfull[2], bempty[2];
-    uint64_t tfull[2], tempty[2];
+    uint8_t sfa_tc[kStages][512];            // 32 rows x 16 B for tcgen05.cp
+    uint8_t sfb_raw[2][kMaxSub * kHeads * 4];
+    uint8_t sfb_tc[2][kMaxPasses][512];
+    float w[2][kMaxSub][kHeads];
+    float* rows[2][kMaxSub];                 // score row of the item's sequence, per problem
+    uint64_t full[kStages], empty[kStages], sfa_ready[kStages];
+    uint64_t bfull[2], bempty[2], sfb_ready[2];
+    uint64_t tfull[kGroups], tempty[kGroups];
     uint64_t drained;
     uint32_t tmem_base;
     int abort;
@@ -78,20 +108,21 @@ static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory beyond the 227 KB pe
 
 
 struct Item {
-    int p, b, t0, t1, n;
+    int s, b, t0, t1, n;
 };
 
 __device__ __forceinline__ bool item_at(const ScanBatch& sb, const MmaScanMaps& mp, int id, Item& it) {
-    const int batch = sb.p[0].cache.batch;
-    const int per_p = batch * mp.chunks;
-    it.p = id / per_p;
-    const int r = id - it.p * per_p;
-    it.b = r / mp.chunks;
-    const int c = r - it.b * mp.chunks;
-    it.n = entries_of(sb.p[it.p].cache, it.b);
+    int s = 0;
+    while (s + 1 < mp.n_sub && id >= mp.sub[s + 1].item0) ++s;
+    const ScanSub& S = mp.sub[s];
+    const int r = id - S.item0;
+    it.s = s;
+    it.b = r / S.chunks;
+    const int c = r - it.b * S.chunks;
+    it.n = entries_of(sb.p[S.prob[0]].cache, it.b);
     const int tiles = (it.n + kTile - 1) / kTile;
-    it.t0 = c * kChunkTiles;
-    it.t1 = min(it.t0 + kChunkTiles, tiles);
+    it.t0 = c * S.chunk;
+    it.t1 = min(it.t0 + S.chunk, tiles);
     return it.t0 < it.t1;
 }
 
@@ -104,24 +135,47 @@ __device__ __forceinline__ bool aborted(Smem& sm) {
     return *reinterpret_cast<volatile int*>(&sm.abort) != 0;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+// 128 rows of 4 scale bytes (one 32-bit word per row) -> the 32x128-bit layout
+// of tcgen05.cp: lane r holds rows r, 32 + r, 64 + r, 96 + r (one per column).
+__device__ __forceinline__ void scales_to_tc(const uint8_t* raw, uint8_t* tc, int lane) {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(raw);
+    reinterpret_cast<uint4*>(tc)[lane] = make_uint4(src[lane], src[32 + lane], src[64 + lane], src[96 + lane]);
+}
+
+// d = a * b + c on two fp32 lanes (each lane an IEEE fma).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    uint64_t d, ua, ub, uc;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ua) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ub) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(uc) : "f"(c.x), "f"(c.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(ua), "l"(ub), "l"(uc));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
     k_scan_mma(const __grid_constant__ ScanBatch sb, const __grid_constant__ MmaScanMaps mp) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int batch = sb.p[0].cache.batch;
-    const int n_items = sb.n * batch * mp.chunks;
+    const int n_items = mp.n_items;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.sfa_ready[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.bfull[i], 1);
-            mbar_init(&sm.bempty[i], 1 + 8);
-            mbar_init(&sm.tfull[i], 1);
-            mbar_init(&sm.tempty[i], 4);  // the four warps of epilogue group i
+            mbar_init(&sm.bempty[i], 1 + kEpiWarps);
+            mbar_init(&sm.sfb_ready[i], 1);
+        }
+        for (int g = 0; g < kGroups; ++g) {
+            mbar_init(&sm.tfull[g], 1);
+            mbar_init(&sm.tempty[g], 8);  // the eight warps of epilogue group g
         }
         mbar_init(&sm.drained, 1);
         sm.abort = 0;
@@ -136,19 +190,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         // Lanes fetch the item's page ids (2 per tile, up to 32) in one round;
-        // lane 0 issues every copy.
+        // one elected lane of the converged warp issues every copy.
         const uint64_t pol_stream = policy_evict_first();
         const uint64_t pol_keep = policy_evict_last();
         if (lane == 0) prefetch_tmap(&mp.queries);
         uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0;
-        int issued[kStages];
-        uint32_t issued_par[kStages];
-        for (int s = 0; s < kStages; ++s) issued[s] = 0, issued_par[s] = 0;
+        uint32_t issued = 0, issued_par = 0;  // per stage: a copy was issued, and its phase
         for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
             Item it;
             if (!item_at(sb, mp, id, it)) continue;
-            const ScanProblem& P = sb.p[it.p];
-            const CacheView& c = P.cache;
+            const ScanSub& S = mp.sub[it.s];
+            const CacheView& c = sb.p[S.prob[0]].cache;
             const int used_pages = (it.n + PAGE - 1) / PAGE;
             const int li = 2 * it.t0 + lane;  // logical page this lane looks up
             int my_pg = -1;
@@ -160,159 +212,201 @@ __global__ void __launch_bounds__(kThreads, 2)
                     atomicOr(c.status, CSA2_DEVERR_PAGE);
             }
             bool stop = false;
-            if (lane == 0) {
-                if (!mbar_wait(&sm.bempty[bslot], bphase ^ 1)) {
-                    raise_abort(sm, c.status);
-                    stop = true;
-                } else {
-                    const int64_t qrow = ((int64_t)it.p * batch + it.b) * kHeads;
-                    mbar_expect_tx(&sm.bfull[bslot], kHeads * 64 + kHeads * 4 + kHeads * 4);
-                    tma_load_2d(sm.b[bslot], &mp.queries, 0, (int)qrow, &sm.bfull[bslot], pol_keep);
-                    bulk_load(sm.sfb_raw[bslot], sb.qs + qrow * ISB, kHeads * 4, &sm.bfull[bslot], pol_keep);
-                    bulk_load(sm.w[bslot], P.w + (int64_t)it.b * kHeads, kHeads * 4, &sm.bfull[bslot], pol_keep);
+            if (!mbar_wait_warp(&sm.bempty[bslot], bphase ^ 1)) {
+                if (lane == 0) raise_abort(sm, c.status);
+                stop = true;
+            } else {
+                if (lane < S.n) sm.rows[bslot][lane] = sb.p[S.prob[lane]].scores + (int64_t)it.b * sb.score_stride;
+                __syncwarp();
+                mbar_expect_tx_w(&sm.bfull[bslot], S.n * (kHeads * 64 + kHeads * 4 + kHeads * 4));
+                for (int j = 0; j < S.n; ++j) {
+                    const int p = S.prob[j];
+                    const int64_t qrow = ((int64_t)p * batch + it.b) * kHeads;
+                    tma_load_2d_w(sm.b[bslot] + j * kHeads * 64, &mp.queries, 0, (int)qrow, &sm.bfull[bslot], pol_keep);
+                    bulk_load_w(sm.sfb_raw[bslot] + j * kHeads * 4, sb.qs + qrow * ISB, kHeads * 4, &sm.bfull[bslot],
+                                pol_keep);
+                    bulk_load_w(sm.w[bslot][j], sb.p[p].w + (int64_t)it.b * kHeads, kHeads * 4, &sm.bfull[bslot],
+                                pol_keep);
                 }
             }
             if (++bslot == 2) bslot = 0, bphase ^= 1;
-            const CUtensorMap* kmap = &mp.keys[mp.src_of[it.p]];
-            for (int t = it.t0; t < it.t1 && !__any_sync(0xffffffffu, stop); ++t) {
+            const CUtensorMap* kmap = &mp.keys[S.src];
+            for (int t = it.t0; t < it.t1 && !stop; ++t) {
                 const int pg0 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0));
                 const int pg1 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0) + 1);
-                if (lane == 0) {
-                    if (!mbar_wait(&sm.empty[stage], sphase ^ 1)) {
-                        raise_abort(sm, c.status);
-                        stop = true;
-                    } else {
-                        const int pg[2] = {pg0, pg1};
-                        const uint32_t bytes = (pg0 >= 0 ? PAGE * (ICB + ISB) : 0) + (pg1 >= 0 ? PAGE * (ICB + ISB) : 0);
-                        if (bytes == 0) {
-                            mbar_arrive(&sm.full[stage]);
-                        } else {
-                            mbar_expect_tx(&sm.full[stage], bytes);
-                            for (int h = 0; h < 2; ++h) {
-                                if (pg[h] < 0) continue;
-                                tma_load_2d(sm.a[stage] + h * PAGE * ICB, kmap, 0, pg[h] * PAGE, &sm.full[stage],
-                                            pol_stream);
-                                bulk_load(sm.sfa_raw[stage] + h * PAGE * ISB,
-                                          c.idx_scales + (int64_t)pg[h] * PAGE * ISB, PAGE * ISB, &sm.full[stage],
-                                          pol_stream);
-                            }
-                        }
-                        issued[stage] = 1;
-                        issued_par[stage] = sphase;
+                if (!mbar_wait_warp(&sm.empty[stage], sphase ^ 1)) {
+                    if (lane == 0) raise_abort(sm, c.status);
+                    stop = true;
+                    break;
+                }
+                const uint32_t bytes = (pg0 >= 0 ? PAGE * (ICB + ISB) : 0) + (pg1 >= 0 ? PAGE * (ICB + ISB) : 0);
+                if (bytes == 0) {
+                    mbar_arrive_w(&sm.full[stage]);
+                } else {
+                    mbar_expect_tx_w(&sm.full[stage], bytes);
+                    if (pg0 >= 0) {
+                        tma_load_2d_w(sm.a[stage], kmap, 0, pg0 * PAGE, &sm.full[stage], pol_stream);
+                        bulk_load_w(sm.sfa_raw[stage], c.idx_scales + (int64_t)pg0 * PAGE * ISB, PAGE * ISB,
+                                    &sm.full[stage], pol_stream);
+                    }
+                    if (pg1 >= 0) {
+                        tma_load_2d_w(sm.a[stage] + PAGE * ICB, kmap, 0, pg1 * PAGE, &sm.full[stage], pol_stream);
+                        bulk_load_w(sm.sfa_raw[stage] + PAGE * ISB, c.idx_scales + (int64_t)pg1 * PAGE * ISB,
+                                    PAGE * ISB, &sm.full[stage], pol_stream);
                     }
                 }
+                issued |= 1u << stage;
+                issued_par = (issued_par & ~(1u << stage)) | (sphase << stage);
                 if (++stage == kStages) stage = 0, sphase ^= 1;
             }
-            if (__any_sync(0xffffffffu, stop)) break;
+            if (stop) break;
         }
         // never leave with copies in flight
         if (lane == 0)
             for (int s = 0; s < kStages; ++s)
-                if (issued[s]) (void)mbar_wait(&sm.full[s], issued_par[s]);
+                if ((issued >> s) & 1u) (void)mbar_wait(&sm.full[s], (issued_par >> s) & 1u);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0, acc = 0, aphase = 0;
-        const uint32_t idesc_lo = idesc_mxf4(kHeads, 0, 0);
-        const uint32_t idesc_hi = idesc_mxf4(kHeads, 2, 2);
         for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
             Item it;
             if (!item_at(sb, mp, id, it)) continue;
-            uint32_t* status = sb.p[it.p].cache.status;
-            if (!mbar_wait_warp(&sm.bfull[bslot], bphase)) { raise_abort(sm, status); break; }
-            {   // query scales -> 32x128b layout: row r holds heads r and 32 + r
-                const uint32_t* src = reinterpret_cast<const uint32_t*>(sm.sfb_raw[bslot]);
-                uint4 v = make_uint4(src[lane], src[32 + lane], 0u, 0u);
-                reinterpret_cast<uint4*>(sm.sfb_tc[bslot])[lane] = v;
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tc_fence_after();
-                    tc_cp_32x128b_x4(tbase + kColSfb + 4 * bslot, smem_desc(sm.sfb_tc[bslot], 16, 128, kLayoutNone));
-                }
-                __syncwarp();
-            }
-            const uint64_t bdesc = smem_desc(sm.b[bslot], 16, 512, kLayoutSw64);
+            const ScanSub& S = mp.sub[it.s];
+            uint32_t* status = sb.p[S.prob[0]].cache.status;
+            const int passes = (S.n + kPass - 1) / kPass;
+            if (!mbar_wait_warp(&sm.sfb_ready[bslot], bphase)) { raise_abort(sm, status); break; }
+            // query scales of each pass -> TMEM (rows = the pass's 128 query rows)
+            tc_fence_after();
+            for (int k = 0; k < passes; ++k)
+                tc_cp_32x128b_x4_w(tbase + kColSfb + (bslot * kMaxPasses + k) * 4,
+                                   smem_desc(sm.sfb_tc[bslot][k], 16, 128, kLayoutNone));
             bool stop = false;
             for (int t = it.t0; t < it.t1; ++t) {
-                if (!mbar_wait_warp(&sm.full[stage], sphase)) { raise_abort(sm, status); stop = true; break; }
-                {   // key scales -> 32x128b layout: row r holds entries r, 32+r, 64+r, 96+r
-                    const uint32_t* src = reinterpret_cast<const uint32_t*>(sm.sfa_raw[stage]);
-                    uint4 v = make_uint4(src[lane], src[32 + lane], src[64 + lane], src[96 + lane]);
-                    reinterpret_cast<uint4*>(sm.sfa_tc[stage])[lane] = v;
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
-                if (!mbar_wait_warp(&sm.tempty[acc], aphase ^ 1)) { raise_abort(sm, status); stop = true; break; }
-                if (lane == 0) {
+                if (!mbar_wait_warp(&sm.sfa_ready[stage], sphase)) { raise_abort(sm, status); stop = true; break; }
+                const uint32_t sfa = tbase + kColSfa + 4 * stage;
+                tc_fence_after();
+                tc_cp_32x128b_x4_w(sfa, smem_desc(sm.sfa_tc[stage], 16, 128, kLayoutNone));
+                const uint64_t adesc = smem_desc(sm.a[stage], 16, 512, kLayoutSw64);
+                for (int k = 0; k < passes; ++k) {
+                    if (!mbar_wait_warp(&sm.tempty[acc], aphase ^ 1)) { raise_abort(sm, status); stop = true; break; }
                     tc_fence_after();
-                    const uint32_t sfa = tbase + kColSfa + 4 * stage;
-                    const uint32_t sfb = tbase + kColSfb + 4 * bslot;
-                    const uint32_t d = tbase + kColAcc + kHeads * acc;
-                    tc_cp_32x128b_x4(sfa, smem_desc(sm.sfa_tc[stage], 16, 128, kLayoutNone));
-                    const uint64_t adesc = smem_desc(sm.a[stage], 16, 512, kLayoutSw64);
+                    const uint32_t n_rows = (uint32_t)min(kPass, S.n - kPass * k) * kHeads;
+                    const uint32_t sfb = tbase + kColSfb + (bslot * kMaxPasses + k) * 4;
+                    const uint32_t d = tbase + kColAcc + 128 * acc;
+                    const uint64_t bdesc = smem_desc(sm.b[bslot] + k * kPass * kHeads * 64, 16, 512, kLayoutSw64);
                     // K = 0..63 (scale bytes 0, 1), then K = 64..127 (bytes 2, 3): +32 B start
-                    tc_mma_mxf4(d, adesc, bdesc, idesc_lo, sfa, sfb, 0u);
-                    tc_mma_mxf4(d, adesc + 2, bdesc + 2, idesc_hi, sfa, sfb, 1u);
-                    tc_commit(&sm.empty[stage]);
-                    tc_commit(&sm.tfull[acc]);
+                    tc_mma_mxf4_w(d, adesc, bdesc, idesc_mxf4(n_rows, 0, 0), sfa, sfb, 0u);
+                    tc_mma_mxf4_w(d, adesc + 2, bdesc + 2, idesc_mxf4(n_rows, 2, 2), sfa, sfb, 1u);
+                    tc_commit_w(&sm.tfull[acc]);
+                    if (++acc == kGroups) acc = 0, aphase ^= 1;
                 }
-                __syncwarp();
+                if (stop) break;
+                tc_commit_w(&sm.empty[stage]);
                 if (++stage == kStages) stage = 0, sphase ^= 1;
-                acc ^= 1;
-                if (acc == 0) aphase ^= 1;
             }
-            if (lane == 0) tc_commit(&sm.bempty[bslot]);
-            __syncwarp();
+            tc_commit_w(&sm.bempty[bslot]);
             if (++bslot == 2) bslot = 0, bphase ^= 1;
             if (stop) break;
         }
         // every tcgen05 operation of this thread has completed before TMEM is freed
-        if (lane == 0) {
-            tc_commit(&sm.drained);
-            (void)mbar_wait(&sm.drained, 0);
-        }
-        __syncwarp();
-    } else {
+        tc_commit_w(&sm.drained);
+        (void)mbar_wait_warp(&sm.drained, 0);
+    } else if (warp < kSfWarp) {
         // ------------------------------------------------------------ epilogue
-        // Group g = (warp - 2) / 4 drains accumulator g, i.e. every other tile.
-        const int grp = (warp - 2) >> 2;
-        const int quad = warp & 3;
+        const int ew = warp - 2;
+        const int grp = ew >> 3;
+        const int jp = (ew >> 2) & 1;     // problem of the pass this warp reads
+        const int quad = warp & 3;        // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;
-        uint32_t bslot = 0, bphase = 0, aphase = 0, tile_no = 0;
+        uint32_t bslot = 0, bphase = 0, aphase = 0, pass_no = 0;
         for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
             Item it;
             if (!item_at(sb, mp, id, it)) continue;
-            const ScanProblem& P = sb.p[it.p];
-            if (!mbar_wait_warp(&sm.bfull[bslot], bphase)) { raise_abort(sm, P.cache.status); break; }
-            const float* w = sm.w[bslot];
-            float* out = P.scores + (int64_t)it.b * sb.score_stride;
+            const ScanSub& S = mp.sub[it.s];
+            const int passes = (S.n + kPass - 1) / kPass;
+            uint32_t* status = sb.p[S.prob[0]].cache.status;
+            if (!mbar_wait_warp(&sm.bfull[bslot], bphase)) { raise_abort(sm, status); break; }
             bool stop = false;
-            for (int t = it.t0; t < it.t1; ++t, ++tile_no) {
-                if ((int)(tile_no & 1u) != grp) continue;
-                if (!mbar_wait_warp(&sm.tfull[grp], aphase)) { raise_abort(sm, P.cache.status); stop = true; break; }
-                aphase ^= 1;
-                tc_fence_after();
-                float v[64];
-                tmem_ld_32x32b_x64(tbase + ((uint32_t)(quad * 32) << 16) + kColAcc + kHeads * grp, v);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.tempty[grp]);
-                float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent chains
+            for (int t = it.t0; t < it.t1 && !stop; ++t) {
+                for (int k = 0; k < passes; ++k, ++pass_no) {
+                    if ((int)(pass_no % kGroups) != grp) continue;
+                    if (!mbar_wait_warp(&sm.tfull[grp], aphase)) { raise_abort(sm, status); stop = true; break; }
+                    aphase ^= 1;
+                    tc_fence_after();
+                    const int j = kPass * k + jp;
+                    if (j < S.n) {
+                        const uint32_t taddr = tbase + ((uint32_t)(quad * 32) << 16) + kColAcc + 128 * grp + 64 * jp;
+                        const float* w = sm.w[bslot][j];
+                        float2 acc2[4];  // eight chains: heads h = 8i + c go to chain c
 #pragma unroll
-                for (int h = 0; h < kHeads; h += 4) {
-                    const float4 w4 = *reinterpret_cast<const float4*>(w + h);
-                    part[0] = fmaf(w4.x, fmaxf(v[h], 0.0f), part[0]);
-                    part[1] = fmaf(w4.y, fmaxf(v[h + 1], 0.0f), part[1]);
-                    part[2] = fmaf(w4.z, fmaxf(v[h + 2], 0.0f), part[2]);
-                    part[3] = fmaf(w4.w, fmaxf(v[h + 3], 0.0f), part[3]);
+                        for (int c = 0; c < 4; ++c) acc2[c] = make_float2(0.0f, 0.0f);
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            float v[32];
+                            tmem_ld_32x32b_x32(taddr + 32 * half, v);
+                            if (half == 1) {
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(&sm.tempty[grp]);
+                            }
+#pragma unroll
+                            for (int h = 0; h < 32; h += 8) {
+                                const float4 wa = *reinterpret_cast<const float4*>(w + 32 * half + h);
+                                const float4 wb = *reinterpret_cast<const float4*>(w + 32 * half + h + 4);
+                                acc2[0] = fma2(make_float2(wa.x, wa.y), make_float2(fmaxf(v[h], 0.0f), fmaxf(v[h + 1], 0.0f)),
+                                               acc2[0]);
+                                acc2[1] = fma2(make_float2(wa.z, wa.w),
+                                               make_float2(fmaxf(v[h + 2], 0.0f), fmaxf(v[h + 3], 0.0f)), acc2[1]);
+                                acc2[2] = fma2(make_float2(wb.x, wb.y),
+                                               make_float2(fmaxf(v[h + 4], 0.0f), fmaxf(v[h + 5], 0.0f)), acc2[2]);
+                                acc2[3] = fma2(make_float2(wb.z, wb.w),
+                                               make_float2(fmaxf(v[h + 6], 0.0f), fmaxf(v[h + 7], 0.0f)), acc2[3]);
+                            }
+                        }
+                        const float s = ((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) +
+                                        ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y));
+                        const int e = t * kTile + row;
+                        if (e < it.n) sm.rows[bslot][j][e] = s;
+                    } else {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm.tempty[grp]);
+                    }
                 }
-                const float s = (part[0] + part[1]) + (part[2] + part[3]);
-                const int e = t * kTile + row;
-                if (e < it.n) out[e] = s;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.bempty[bslot]);
             if (++bslot == 2) bslot = 0, bphase ^= 1;
+            if (stop) break;
+        }
+    } else {
+        // ------------------------------------------------------------ scale warp
+        uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0;
+        for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
+            Item it;
+            if (!item_at(sb, mp, id, it)) continue;
+            const ScanSub& S = mp.sub[it.s];
+            uint32_t* status = sb.p[S.prob[0]].cache.status;
+            const int passes = (S.n + kPass - 1) / kPass;
+            if (!mbar_wait_warp(&sm.bfull[bslot], bphase)) { if (lane == 0) raise_abort(sm, status); break; }
+            for (int k = 0; k < passes; ++k) scales_to_tc(sm.sfb_raw[bslot] + k * 512, sm.sfb_tc[bslot][k], lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sfb_ready[bslot]);
+            if (++bslot == 2) bslot = 0, bphase ^= 1;
+            bool stop = false;
+            for (int t = it.t0; t < it.t1; ++t) {
+                if (!mbar_wait_warp(&sm.full[stage], sphase)) {
+                    if (lane == 0) raise_abort(sm, status);
+                    stop = true;
+                    break;
+                }
+                scales_to_tc(sm.sfa_raw[stage], sm.sfa_tc[stage], lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sfa_ready[stage]);
+                if (++stage == kStages) stage = 0, sphase ^= 1;
+            }
             if (stop) break;
         }
     }
@@ -382,12 +476,13 @@ cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st) {
     MmaScanMaps mp;
     std::memset(&mp, 0, sizeof(mp));
     const int batch = sb.p[0].cache.batch;
+    // distinct caches -> key maps; problems of one cache -> subsets of <= kMaxSub
     int srcs = 0;
     const uint8_t* seen[kMaxSources];
-    int cap = 0;
+    int src_of[kMaxProblems];
+    int cap_tiles[kMaxSources];
     for (int i = 0; i < sb.n; ++i) {
         const CacheView& c = sb.p[i].cache;
-        cap = max(cap, c.max_pages * PAGE);
         int j = 0;
         for (; j < srcs; ++j)
             if (seen[j] == c.idx_codes) break;
@@ -395,16 +490,46 @@ cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st) {
             seen[srcs] = c.idx_codes;
             if (!make_rows64_map(&mp.keys[srcs], c.idx_codes, (uint64_t)c.num_pages * PAGE, PAGE))
                 return cudaErrorInvalidValue;
+            cap_tiles[srcs] = (c.max_pages * PAGE + kTile - 1) / kTile;
             ++srcs;
         }
-        mp.src_of[i] = j;
+        src_of[i] = j;
+    }
+    for (int j = 0; j < srcs; ++j) {
+        int members[kMaxProblems], m = 0;
+        for (int i = 0; i < sb.n; ++i)
+            if (src_of[i] == j) members[m++] = i;
+        // split into near-equal subsets of at most kMaxSub problems
+        const int parts = (m + kMaxSub - 1) / kMaxSub;
+        for (int q = 0, i0 = 0; q < parts; ++q) {
+            const int cnt = (m - i0) / (parts - q);
+            ScanSub& S = mp.sub[mp.n_sub++];
+            S.src = j;
+            S.n = cnt;
+            for (int k = 0; k < cnt; ++k) S.prob[k] = (int8_t)members[i0 + k];
+            i0 += cnt;
+        }
+    }
+    // Tiles per work item: about 64 tile-problems of work each (so subsets of
+    // different sizes cost about the same per item), fewer when the items would
+    // not fill the grid a few times over.
+    const int grid_max = sm_count();
+    int items = 0;
+    for (int base = 64;; base /= 2) {
+        items = 0;
+        for (int s = 0; s < mp.n_sub; ++s) {
+            ScanSub& S = mp.sub[s];
+            S.chunk = std::max(2, std::min(kMaxChunk, base / S.n));
+            S.chunks = (cap_tiles[S.src] + S.chunk - 1) / S.chunk;
+            S.item0 = items;
+            items += batch * S.chunks;
+        }
+        if (items >= 3 * grid_max || base <= 4) break;
     }
     if (!make_rows64_map(&mp.queries, sb.qc, (uint64_t)sb.n * batch * kHeads, kHeads))
         return cudaErrorInvalidValue;
-    const int tiles = (cap + kTile - 1) / kTile;
-    mp.chunks = (tiles + kChunkTiles - 1) / kChunkTiles;
-    const long n_items = (long)sb.n * batch * mp.chunks;
-    const int grid = (int)std::min<long>(n_items, 2L * sm_count());
+    mp.n_items = items;
+    const int grid = std::min(items, grid_max);
     const size_t smem = sizeof(Smem) + 1024;
     static const bool attr = [smem] {
         cudaFuncSetAttribute(k_scan_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

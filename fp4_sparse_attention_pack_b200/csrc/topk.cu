@@ -3,7 +3,7 @@
 // Scores map to order-preserving uint32 keys; the K largest are kept, equal
 // scores lower index first, and written in increasing index order.
 //
-// One CTA of 1024 threads per (problem, sequence):
+// One CTA of 512 threads per (problem, sequence), four CTAs per SM:
 //   1. Threshold guess: 2,048 strided samples of the row; an exact radix select
 //      in shared memory finds the sample key ranked ~2K * 2048 / n, so that
 //      about 2K of the n scores lie at or above it.
@@ -23,10 +23,11 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kThreads = 1024;
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
 constexpr int kSamples = 2048;
-constexpr int kCap = 12288;
-constexpr int kRun = 16;  // contiguous scores per thread per pass
+constexpr int kCap = 4096;  // candidates kept in shared memory (the guess targets about 2K + 1 %)
+constexpr int kRun = 8;   // contiguous scores per thread per pass
 
 struct TopkSmem {
     uint32_t key[kCap];
@@ -51,7 +52,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* excl) {
     if (lane == 31) s_warp[wid] = x;
     __syncthreads();
     if (wid == 0) {
-        int t = s_warp[lane];
+        int t = lane < kWarps ? s_warp[lane] : 0;
         int u = t;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -160,7 +161,7 @@ __device__ void emit_topk(KeyAt key_at, IdxAt idx_at, int cnt, uint32_t kth, int
     }
 }
 
-__global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanBatch sb) {
+__global__ void __launch_bounds__(kThreads, 4) k_topk(const __grid_constant__ ScanBatch sb) {
     extern __shared__ uint8_t smem_raw[];
     TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
     const ScanProblem& P = sb.p[blockIdx.y];

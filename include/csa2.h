@@ -313,6 +313,17 @@ int csa2_layer_step_profiled(const csa2_model* model, const csa2_step_in* in,
                              const csa2_step_out* out, void* ws, size_t ws_bytes,
                              csa2_stream stream, void* const* events);
 
+/*
+ * Number of kernel launches one csa2_layer_step(model, in, ...) call enqueues
+ * on the current device (the measurement variant adds none): the window
+ * append, two for the cache write when any source takes a token, three for the
+ * indexer (query quantisation, scan, Top-K) when any layer scans, and one or two
+ * for attention (a second one combines split tiles when there are fewer
+ * (layer, sequence) pairs than SMs).  Returns a negative csa2_status when the
+ * model table is invalid or `in` is NULL.  Enqueues nothing.
+ */
+int csa2_layer_step_launches(const csa2_model* model, const csa2_step_in* in);
+
 #ifdef __cplusplus
 }
 #endif

@@ -299,9 +299,19 @@ def test_window_append_ring(csa):
 
 # ---------------------------------------------------------------- layer step
 
-@pytest.mark.parametrize("table_name,H_idx", [("alternating", 16), ("pages", 16), ("alternating", 64)])
+def _reindex16_table():
+    """16 layers over one ratio-2 source: Full, 13 Reindex, 2 Reuse.  Fourteen
+    scans read one cache, more than one grouped work item holds (two subsets of
+    seven problems, each ending in a single-problem MMA pass)."""
+    mode = (W.FULL,) + (W.REINDEX,) * 13 + (W.REUSE,) * 2
+    return W.ModeTable(mode, (0,) * 16, tuple(range(14)) + (13, 13), (2,))
+
+
+@pytest.mark.parametrize("table_name,H_idx", [("alternating", 16), ("pages", 16), ("alternating", 64),
+                                              ("pages", 64), ("reindex16", 64)])
 def test_layer_step_parity(csa, table_name, H_idx):
-    table = W.schedule_alternating_40() if table_name == "alternating" else W.schedule_pages_40()
+    table = {"alternating": W.schedule_alternating_40, "pages": W.schedule_pages_40,
+             "reindex16": _reindex16_table}[table_name]()
     wl = W.Workload("small40", 7, 2, 601, table, 8, H_idx, 64, 3)
     dm = csa.engine.DecodeModel(wl, DEV, page_seed=21)
     dm.fill(chunk_tokens=256)
