@@ -10,26 +10,22 @@
 //   P^T = exp(scale * S^T - m_head)                    (fp16, per item lane)
 //   O^T[4 x 128 latent x 64 heads] += Items^T . P^T    (M = 128, N = 64, K = 128)
 //
-// A tile is consumed as eight slabs of 64 latent channels (128 rows x 128 B,
-// 128-byte swizzle), each read as the K-major A operand of S^T and, two at a
-// time, as the MN-major A operand of O^T.  The running per-head maximum is only
-// moved when a tile's maximum exceeds it by more than 8 (so p <= e^8 fits
-// fp16), which makes the O rescale (TMEM load, scale, store) rare.  Heads are
-// padded to 64.
+// One shared-memory image of the tile serves both MMAs: 128-byte-swizzled
+// slabs of 64 latent channels, read as the K-major A operand of S^T and as the
+// MN-major A operand of O^T.  The running per-head maximum is only moved when
+// a tile's maximum exceeds it by more than 8 (so p <= e^8 fits fp16), which
+// makes the O rescale (TMEM load, scale, store) rare.  Heads are padded to 64.
 //
-// Warp-specialised CTA (416 threads, one unit = (problem, sequence, split)):
-//   warps 8-11  slab producers, one item row per thread: dequantise the row's
-//               cache entry (16-byte loads issued three slabs ahead) or convert
-//               its window token (slab boxes by TMA, 3-D tensor map per window,
-//               started four slabs ahead) into a ring of eight 16 KB slab slots;
-//   warp 12     MMA issuer (one elected lane of the converged warp) in the
-//               order S(0), S(1), O(0), S(2), O(1), ..., O(last), so that the
-//               softmax of tile t overlaps the S MMAs of tile t + 1; the slabs of
-//               a tile are produced twice (once for S, once for O);
-//   warps 0-7   softmax (two per TMEM lane quadrant, 32 heads each) into a
-//               double-buffered S^T, P^T to shared memory, rescale of O^T, and
-//               the final normalised write of O.
-// Every wait is bounded; a timeout sets CSA2_DEVERR_TIMEOUT and the CTA drains.
+// CTA = 256 threads, one unit (problem, sequence, split of tiles) per CTA.
+// Gather: the unit's selected entries and window are prefetched into L2 first;
+// window rows arrive by TMA (a 3-D tensor map per window, 128-byte swizzle, one
+// box per slab, so they land directly in the slab layout and are converted
+// bf16 -> fp16 in place); cache entries are loaded with 16-byte loads (eight
+// lanes per entry row) and dequantised in registers, the chunk order staggered
+// per lane so the swizzled stores are free of bank conflicts.  Warp 0 issues the MMAs (one
+// elected lane, the warp converged); all eight
+// warps run the softmax (two per TMEM lane quadrant, 32 heads each) and
+// rescale / write O.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -50,36 +46,30 @@ using namespace sm100;
 
 constexpr int kT = 128;            // items per tile (MMA M of S^T)
 constexpr int kHp = 64;            // heads, padded (MMA N)
-constexpr int kSlots = 8;          // slab ring
-constexpr int kSlabBytes = kT * 128;
-constexpr int kSoftWarps = 8;      // warps 0-7
-constexpr int kProdWarp0 = 8;      // warps 8-11
-constexpr int kMmaWarp = 12;
-constexpr int kThreads = 32 * 13;
-constexpr int kMaxUnitTiles = (CSA2_MAX_K + WIN + kT - 1) / kT;
+constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // S^T: 2 x 64 columns
-constexpr uint32_t kColO = 128;    // O^T: 4 x 64 columns
+constexpr uint32_t kColS = 0;      // S^T: 64 columns
+constexpr uint32_t kColO = 64;     // O^T: 4 x 64 columns
 constexpr float kRescaleGap = 8.0f;
-constexpr int kRowEmpty = -1, kRowWindow = -2;  // lookup codes (else: entry row in the pools)
 
 struct AttnMaps {
     CUtensorMap win[kMaxProblems];  // window [batch][128][512] bf16, box 64 x 128 x 1, SW128
 };
 
 struct __align__(1024) Smem {
-    uint8_t slab[kSlots][kSlabBytes];  // 128 rows x 128 B (SW128) each
-    uint8_t q[8][kHp * 128];           // 8 slabs x 64 rows x 128 B (SW128)
-    uint8_t p[kT * 128];               // P^T: 128 item rows x 64 heads fp16 (SW128)
-    int32_t lk[kMaxUnitTiles][kT];     // per unit tile and row: entry row, kRowWindow or kRowEmpty
-    float red_max[4][kHp];             // per-quadrant partial max
-    float red_sum[4][kHp];             // per-quadrant partial sum
+    uint8_t items[8][kT * 128];    // 8 slabs x 128 rows x 128 B (SW128)
+    uint8_t q[8][kHp * 128];       // 8 slabs x 64 rows x 128 B (SW128)
+    uint8_t p[kT * 128];           // P^T: 128 item rows x 64 heads fp16 (SW128)
+    float red[4][kHp];             // per-quadrant partial max / sum
     float m_used[kHp];
     float l[kHp];
     float alpha[kHp];
-    int rescale[2];                    // per head warp: some head's maximum moved
-    uint64_t slot_full[kSlots], slot_empty[kSlots], tma_bar[kSlots];
-    uint64_t s_full[2], s_empty[2], p_full, o_done, drained;
+    int kind[2][kT];               // per tile buffer: 0 empty, 1 cache entry, 2 window token
+    int64_t src_row[2][kT];        // entry row in the pools
+    int n_entries[2];
+    int has_window[2];
+    uint64_t bar;                  // MMA completion
+    uint64_t wbar;                 // window TMA
     uint32_t tmem_base;
 };
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory beyond the 227 KB per-block limit");
@@ -138,58 +128,6 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&v)[N]) {
     }
 }
 
-// All 256 softmax threads meet (named barrier 1); returns the OR of pred over them.
-__device__ __forceinline__ bool soft_sync_or(bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.or.pred q, 1, 256, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred)
-        : "memory");
-    return r != 0;
-}
-
-__device__ __forceinline__ void soft_sync() { asm volatile("barrier.cta.sync 1, 256;" ::: "memory"); }
-
-// Dequantise one entry row of slab j: 32 code bytes (64 E2M1 values, channel 2i
-// in the low nibble) and 4 E4M3 scale bytes (one per 16 channels) -> fp16.
-__device__ __forceinline__ void dequant_row(uint8_t* slab, int r, uint4 c0, uint4 c1, uint32_t sc) {
-    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-    for (int c2 = 0; c2 < 4; ++c2) {  // chunks 2*c2, 2*c2+1 share scale byte c2
-        const __half2 s2 = __float2half2_rn(e4m3_decode_pos((sc >> (8 * c2)) & 0xFFu));
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * c2 + cc;
-            uint4 o;
-            uint32_t* os = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t h = e2m1x2_to_h2((cw[c] >> (8 * k)) & 0xFFu);
-                const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&h), s2);
-                os[k] = *reinterpret_cast<const uint32_t*>(&v);
-            }
-            *reinterpret_cast<uint4*>(slab + sw128(r, c)) = o;
-        }
-    }
-}
-
-// Step s of a unit with n tiles: S(0), S(1), O(0), S(2), O(1), ..., S(n-1), O(n-2), O(n-1).
-__device__ __forceinline__ void unit_step(int s, int n, int& tile, bool& is_s) {
-    if (s == 0) {
-        tile = 0, is_s = true;
-    } else if (s == 2 * n - 1) {
-        tile = n - 1, is_s = false;
-    } else if (s & 1) {
-        tile = (s + 1) >> 1, is_s = true;
-    } else {
-        tile = (s >> 1) - 1, is_s = false;
-    }
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_mma(const __grid_constant__ AttnBatch ab, const __grid_constant__ AttnMaps maps, int splits,
                int tiles_per_split) {
@@ -206,31 +144,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int H = ab.H;
     const int n_tiles = (K + WIN + kT - 1) / kT;
     const int t_begin = split * tiles_per_split;
-    const int nt = max(0, min(n_tiles, t_begin + tiles_per_split) - t_begin);  // tiles of this unit
+    const int t_end = min(n_tiles, t_begin + tiles_per_split);
 
     if (tid == 0) {
-        for (int i = 0; i < kSlots; ++i) {
-            mbar_init(&sm.slot_full[i], 4);  // the four producer warps
-            mbar_init(&sm.slot_empty[i], 1);
-            mbar_init(&sm.tma_bar[i], 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.s_full[i], 1);
-            mbar_init(&sm.s_empty[i], kSoftWarps);
-        }
-        mbar_init(&sm.p_full, kSoftWarps);
-        mbar_init(&sm.o_done, 1);
-        mbar_init(&sm.drained, 1);
+        mbar_init(&sm.bar, 1);
+        mbar_init(&sm.wbar, 1);
+        sm.n_entries[0] = sm.n_entries[1] = 0;
+        sm.has_window[0] = sm.has_window[1] = 0;
         fence_mbar_init();
         prefetch_tmap(&maps.win[prob]);
     }
-    if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
+    if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
     if (tid < kHp) {
         sm.m_used[tid] = -INFINITY;
         sm.l[tid] = 0.0f;
     }
     // Q -> fp16 slabs (rows >= H are zero): cp.async in place, then convert.
-    if (warp < 8) {
+    {
         const int j = warp;
         for (int h = lane; h < kHp; h += 32) {
             if (h < H) {
@@ -248,312 +178,305 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wcount = P.win_count[b];
     const int wlen = wcount < WIN ? (wcount < 0 ? 0 : wcount) : WIN;
     const int n = (K > 0) ? entries_of(P.cache, b) : 0;
-    // Where every item of the unit comes from, and its entries into L2 now.
-    for (int i = tid; i < nt * kT; i += kThreads) {
-        const int u = i / kT, r = i - u * kT;
-        const int pos = (t_begin + u) * kT + r;
-        int32_t code = kRowEmpty;
-        if (pos < K) {
+    // Bring this unit's selected entries and window ring into L2 now, so that
+    // every tile's gather below is served from L2 rather than waiting on DRAM.
+    {
+        const int p_end = min(K, t_end * kT);
+        for (int pos = t_begin * kT + tid; pos < p_end; pos += kThreads) {
             const int e = P.idx[(int64_t)b * K + pos];
             if (e >= 0 && e < n) {
                 const int pg = page_of(P.cache, b, e);
                 if (pg >= 0) {
-                    code = pg * PAGE + (e % PAGE);
-                    bulk_prefetch_l2(P.cache.main_codes + (int64_t)code * MCB, MCB);
-                    bulk_prefetch_l2(P.cache.main_scales + (int64_t)code * MSB, MSB);
+                    const int64_t ent = (int64_t)pg * PAGE + (e % PAGE);
+                    bulk_prefetch_l2(P.cache.main_codes + ent * MCB, MCB);
+                    bulk_prefetch_l2(P.cache.main_scales + ent * MSB, MSB);
                 }
             }
-        } else if (pos - K < wlen) {
-            code = kRowWindow;
         }
-        sm.lk[u][r] = code;
+        if (tid == 0 && t_end * kT > K && wlen > 0)
+            bulk_prefetch_l2(P.win + (int64_t)b * WIN * D, (uint32_t)wlen * D * 2);
     }
-    if (tid == 0 && nt > 0 && (t_begin + nt) * kT > K && wlen > 0)
-        bulk_prefetch_l2(P.win + (int64_t)b * WIN * D, (uint32_t)wlen * D * 2);
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
+    uint32_t phase = 0, wphase = 0;
+    bool o_init = false;
     bool timed_out = false;
 
-    if (warp >= kProdWarp0 && warp < kMmaWarp) {
-        // ------------------------------------------------------------ producers
-        const int r = tid - kProdWarp0 * 32;  // item row of this thread
-        const bool issuer = warp == kProdWarp0;
-        uint32_t tma_par = 0, tma_pending = 0;
-        const int n_prod = 16 * nt;
-        auto prod_at = [&](int q, int& u, int& j) {
-            bool is_s;
-            unit_step(q >> 3, nt, u, is_s);
-            j = q & 7;
-        };
-        auto load_raw = [&](int q, uint4& c0, uint4& c1, uint32_t& sc) {
-            int u, j;
-            prod_at(q, u, j);
-            const int32_t code = sm.lk[u][r];
-            if (code >= 0) {
-                const uint4* cs = reinterpret_cast<const uint4*>(P.cache.main_codes + (int64_t)code * MCB + 32 * j);
-                c0 = __ldg(cs);
-                c1 = __ldg(cs + 1);
-                sc = __ldg(reinterpret_cast<const uint32_t*>(P.cache.main_scales + (int64_t)code * MSB + 4 * j));
+    const uint32_t idesc_s = idesc_f16(128, kHp, 0, 0, 0);
+    const uint32_t idesc_o = idesc_f16(128, kHp, 0, 1, 1);
+    const uint64_t desc_items = smem_desc(sm.items[0], 16, 1024, kLayoutSw128);
+    const uint64_t desc_q = smem_desc(sm.q[0], 16, 1024, kLayoutSw128);
+    const uint64_t desc_vt = smem_desc(sm.items[0], 16384, 1024, kLayoutSw128);
+    const uint64_t desc_p = smem_desc(sm.p, 16384, 1024, kLayoutSw128);
+
+    // Where each item of tile t comes from (one thread per item), into buffer buf.
+    auto lookup = [&](int t, int buf) {
+        if (tid < kT) {
+            const int pos = t * kT + tid;
+            int kind = 0;
+            int64_t row = -1;
+            if (pos < K) {
+                const int e = P.idx[(int64_t)b * K + pos];
+                if (e >= 0 && e < n) {
+                    const int pg = page_of(P.cache, b, e);
+                    if (pg >= 0) {
+                        kind = 1;
+                        row = (int64_t)pg * PAGE + (e % PAGE);
+                    }
+                }
+            } else if (pos - K < wlen) {
+                kind = 2;
+            }
+            sm.kind[buf][tid] = kind;
+            sm.src_row[buf][tid] = row;
+            const unsigned ent = __ballot_sync(0xffffffffu, kind == 1);
+            const unsigned win = __ballot_sync(0xffffffffu, kind == 2);
+            if (lane == 0) {
+                if (ent) atomicAdd(&sm.n_entries[buf], __popc(ent));
+                if (win) sm.has_window[buf] = 1;
+            }
+        }
+    };
+    // Packed bytes of the tile's cache entries: warp = slab j, lane = rows lane + 32 i.
+    uint4 raw0[4], raw1[4];
+    uint32_t raws[4];
+    auto load_entries = [&](int buf) {
+        const int j = warp;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = lane + 32 * i;
+            if (sm.kind[buf][r] == 1) {
+                const int64_t ent = sm.src_row[buf][r];
+                const uint4* cs = reinterpret_cast<const uint4*>(P.cache.main_codes + ent * MCB + 32 * j);
+                raw0[i] = __ldg(cs);
+                raw1[i] = __ldg(cs + 1);
+                raws[i] = __ldg(reinterpret_cast<const uint32_t*>(P.cache.main_scales + ent * MSB + 4 * j));
             } else {
-                c0 = c1 = make_uint4(0, 0, 0, 0);
-                sc = 0;
-            }
-        };
-        auto window_tile = [&](int u) {
-            const int t = t_begin + u;
-            return (t * kT + kT > K) && (t * kT < K + wlen);
-        };
-        // Window boxes: the issuing warp acquires slots and starts their TMA loads
-        // kTmaAhead productions ahead of the one being built.
-        constexpr int kTmaAhead = 4;
-        auto acquire = [&](int qa) -> bool {
-            int u, j;
-            prod_at(qa, u, j);
-            const int slot = qa & (kSlots - 1);
-            if (!mbar_wait_warp(&sm.slot_empty[slot], ((qa >> 3) & 1) ^ 1)) return false;
-            if (window_tile(u)) {
-                mbar_expect_tx_w(&sm.tma_bar[slot], kSlabBytes);
-                tma_load_3d_w(sm.slab[slot], &maps.win[prob], 64 * j, (t_begin + u) * kT - K, b, &sm.tma_bar[slot]);
-                tma_pending |= 1u << slot;
-            }
-            return true;
-        };
-        if (issuer)
-            for (int qa = 0; qa < kTmaAhead && qa < n_prod && !timed_out; ++qa) timed_out = !acquire(qa);
-        // Entry bytes: three productions ahead in registers.
-        uint4 ra0[3], ra1[3];
-        uint32_t rsc[3];
-#pragma unroll
-        for (int i = 0; i < 3; ++i) {
-            if (i < n_prod) {
-                load_raw(i, ra0[i], ra1[i], rsc[i]);
-            } else {
-                ra0[i] = ra1[i] = make_uint4(0, 0, 0, 0);
-                rsc[i] = 0;
+                raw0[i] = raw1[i] = make_uint4(0, 0, 0, 0);
+                raws[i] = 0;
             }
         }
-        for (int q = 0; q < n_prod && !timed_out; ++q) {
-            const uint4 c0 = ra0[0], c1 = ra1[0];
-            const uint32_t sc = rsc[0];
-            ra0[0] = ra0[1], ra1[0] = ra1[1], rsc[0] = rsc[1];
-            ra0[1] = ra0[2], ra1[1] = ra1[2], rsc[1] = rsc[2];
-            if (q + 3 < n_prod) load_raw(q + 3, ra0[2], ra1[2], rsc[2]);
-            if (issuer && q + kTmaAhead < n_prod && !acquire(q + kTmaAhead)) { timed_out = true; break; }
-            int u, j;
-            prod_at(q, u, j);
-            const int slot = q & (kSlots - 1);
-            if (!mbar_wait_warp(&sm.slot_empty[slot], ((q >> 3) & 1) ^ 1)) { timed_out = true; break; }
-            uint8_t* slab = sm.slab[slot];
-            if (window_tile(u)) {
-                if (!mbar_wait_warp(&sm.tma_bar[slot], (tma_par >> slot) & 1u)) { timed_out = true; break; }
-                tma_par ^= 1u << slot;
-                tma_pending &= ~(1u << slot);
-            }
-            const int32_t code = sm.lk[u][r];
-            if (code >= 0)
-                dequant_row(slab, r, c0, c1, sc);
-            else if (code == kRowWindow)
-                bf16_row_to_f16(slab, r);
-            else
-                zero_row(slab, r);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.slot_full[slot]);
+    };
+
+    int buf = 0;
+    if (t_begin < t_end) {
+        lookup(t_begin, 0);
+        __syncthreads();
+        load_entries(0);
+    }
+    for (int t = t_begin; t < t_end && !timed_out; ++t, buf ^= 1) {
+        const bool has_window = sm.has_window[buf] != 0;
+        // ---- window rows by TMA, one 64-channel box per slab (O of the previous
+        // tile has completed, so the item buffer is free)
+        if (warp == 0 && has_window) {
+            mbar_expect_tx_w(&sm.wbar, 8 * kT * 128);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) tma_load_3d_w(sm.items[j], &maps.win[prob], 64 * j, t * kT - K, b, &sm.wbar);
         }
-        // a window box still in flight lands before the CTA moves on
-        if (issuer && lane == 0)
-            for (int i = 0; i < kSlots; ++i)
-                if ((tma_pending >> i) & 1u) (void)mbar_wait(&sm.tma_bar[i], (tma_par >> i) & 1u);
-        __syncwarp();
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer
-        const uint32_t idesc_s = idesc_f16(128, kHp, 0, 0, 0);
-        const uint32_t idesc_o = idesc_f16(128, kHp, 0, 1, 1);
-        const uint64_t desc_slab0 = smem_desc(sm.slab[0], 16, 1024, kLayoutSw128);
-        const uint64_t desc_vt0 = smem_desc(sm.slab[0], kSlabBytes, 1024, kLayoutSw128);
-        const uint64_t desc_q = smem_desc(sm.q[0], 16, 1024, kLayoutSw128);
-        const uint64_t desc_p = smem_desc(sm.p, kSlabBytes, 1024, kLayoutSw128);
-        int q = 0;
-        for (int st = 0; st < 2 * nt && !timed_out; ++st) {
-            int u;
-            bool is_s;
-            unit_step(st, nt, u, is_s);
-            if (is_s) {
-                if (u >= 2 && !mbar_wait_warp(&sm.s_empty[u & 1], ((u - 2) >> 1) & 1)) { timed_out = true; break; }
-                const uint32_t d = tbase + kColS + 64 * (u & 1);
-                for (int j = 0; j < 8; ++j, ++q) {
-                    const int slot = q & (kSlots - 1);
-                    if (!mbar_wait_warp(&sm.slot_full[slot], (q >> 3) & 1)) { timed_out = true; break; }
-                    tc_fence_after();
-                    const uint64_t da = desc_slab0 + (uint64_t)((slot * kSlabBytes) >> 4);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)  // 16 latent channels per MMA
-                        tc_mma_f16_w(d, da + 2 * k, desc_q + (uint64_t)((j * kHp * 128 + 32 * k) >> 4), idesc_s,
-                                     (j | k) ? 1u : 0u);
-                    tc_commit_w(&sm.slot_empty[slot]);
-                }
-                if (timed_out) break;
-                tc_commit_w(&sm.s_full[u & 1]);
-            } else {
-                if (!mbar_wait_warp(&sm.p_full, u & 1)) { timed_out = true; break; }
-                for (int c = 0; c < 4; ++c, q += 2) {
-                    const int slot = q & (kSlots - 1);  // slabs 2c, 2c+1 sit in adjacent slots
-                    if (!mbar_wait_warp(&sm.slot_full[slot], (q >> 3) & 1) ||
-                        !mbar_wait_warp(&sm.slot_full[slot + 1], ((q + 1) >> 3) & 1)) {
-                        timed_out = true;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t da = desc_vt0 + (uint64_t)((slot * kSlabBytes) >> 4);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)  // 16 items per MMA
-                        tc_mma_f16_w(tbase + kColO + 64 * c, da + (uint64_t)((2048 * i) >> 4),
-                                     desc_p + (uint64_t)((2048 * i) >> 4), idesc_o, (u > 0 || i > 0) ? 1u : 0u);
-                    tc_commit_w(&sm.slot_empty[slot]);
-                    tc_commit_w(&sm.slot_empty[slot + 1]);
-                }
-                if (timed_out) break;
-                tc_commit_w(&sm.o_done);
-            }
+        // ---- cache entries (bytes already in registers): warp = slab, lane = row.
+        // The window boxes cover all 128 rows, so they must land first.
+        if (has_window) {
+            if (!mbar_wait(&sm.wbar, wphase)) timed_out = true;
+            wphase ^= 1;
         }
-        // every tcgen05 operation of this warp has completed before TMEM is freed
-        tc_commit_w(&sm.drained);
-        (void)mbar_wait_warp(&sm.drained, 0);
-    } else {
-        // ------------------------------------------------------------ softmax + output
-        const int quad = warp & 3, hh = warp >> 2;
-        const int row = quad * 32 + lane;
-        for (int u = 0; u < nt; ++u) {
-            bool ok_wait = mbar_wait(&sm.s_full[u & 1], (u >> 1) & 1);
-            if (soft_sync_or(!ok_wait)) { timed_out = true; break; }
-            tc_fence_after();
-            const uint32_t s_addr = tbase + ((uint32_t)(quad * 32) << 16) + kColS + 64 * (u & 1) + 32 * hh;
-            const bool ok = sm.lk[u][row] != kRowEmpty;
-            {
-                float v[32];
-                tmem_ld_32x32b_x32(s_addr, v);
+        {
+            const int j = warp;
 #pragma unroll
-                for (int h = 0; h < 32; ++h) v[h] = ok ? v[h] * ab.scale : -INFINITY;
-                warp_reduce_scatter<true, 32>(v);
-                sm.red_max[quad][32 * hh + lane] = v[0];
-            }
-            soft_sync();
-            if (tid < kHp) {
-                const float mt = fmaxf(fmaxf(sm.red_max[0][tid], sm.red_max[1][tid]),
-                                       fmaxf(sm.red_max[2][tid], sm.red_max[3][tid]));
-                const float mo = sm.m_used[tid];
-                float a = 1.0f;
-                bool rs = false;
-                if (mt > mo + kRescaleGap || (mo == -INFINITY && mt != -INFINITY)) {
-                    a = (mo == -INFINITY) ? 0.0f : expf(mo - mt);
-                    sm.m_used[tid] = mt;
-                    rs = u > 0 && mo != -INFINITY;
-                }
-                sm.alpha[tid] = a;
-                const unsigned any = __ballot_sync(0xffffffffu, rs);
-                if (lane == 0) sm.rescale[warp] = any ? 1 : 0;
-            }
-            // P^T and O^T of the previous tile are in use until its O MMAs complete
-            ok_wait = (u == 0) || mbar_wait(&sm.o_done, (u - 1) & 1);
-            if (soft_sync_or(!ok_wait)) { timed_out = true; break; }
-            tc_fence_after();
-            const bool rescale = (sm.rescale[0] | sm.rescale[1]) != 0;
-            // ---- P^T = exp(s - m) in fp16 (S reloaded from TMEM), sums of the rounded p
-            {
-                float v[32];
-                tmem_ld_32x32b_x32(s_addr, v);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.s_empty[u & 1]);
+            for (int i = 0; i < 4; ++i) {
+                const int r = lane + 32 * i;
+                const int kind = sm.kind[buf][r];
+                if (kind == 2) {
+                    bf16_row_to_f16(sm.items[j], r);
+                } else if (kind == 0) {
+                    zero_row(sm.items[j], r);
+                } else {
+                    const uint32_t cw[8] = {raw0[i].x, raw0[i].y, raw0[i].z, raw0[i].w,
+                                            raw1[i].x, raw1[i].y, raw1[i].z, raw1[i].w};
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint4 o;
-                    uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+                    for (int c2 = 0; c2 < 4; ++c2) {  // chunks 2*c2, 2*c2+1 share scale byte c2
+                        const __half2 s2 = __float2half2_rn(e4m3_decode_pos((raws[i] >> (8 * c2)) & 0xFFu));
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int h = 8 * c + 2 * k;
-                        const float p0 = ok ? __expf(v[h] * ab.scale - sm.m_used[32 * hh + h]) : 0.0f;
-                        const float p1 = ok ? __expf(v[h + 1] * ab.scale - sm.m_used[32 * hh + h + 1]) : 0.0f;
-                        const __half2 hv = __floats2half2_rn(p0, p1);
-                        const float2 back = __half22float2(hv);
-                        v[h] = back.x;
-                        v[h + 1] = back.y;
-                        os[k] = *reinterpret_cast<const uint32_t*>(&hv);
-                    }
-                    *reinterpret_cast<uint4*>(sm.p + sw128(row, 4 * hh + c)) = o;
-                }
-                warp_reduce_scatter<false, 32>(v);
-                sm.red_sum[quad][32 * hh + lane] = v[0];
-            }
-            // ---- rescale O^T where a head's reference maximum moved
-            if (rescale) {
-                for (int c = hh * 2; c < hh * 2 + 2; ++c) {
-                    const uint32_t ta = tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * c;
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int c = 2 * c2 + cc;
+                            uint4 o;
+                            uint32_t* os = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float o[32];
-                        tmem_ld_32x32b_x32(ta + 32 * half, o);
-#pragma unroll
-                        for (int h = 0; h < 32; ++h) o[h] *= sm.alpha[32 * half + h];
-                        tmem_st_32x32b_x32(ta + 32 * half, o);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            soft_sync();
-            if (tid < kHp)
-                sm.l[tid] = sm.l[tid] * sm.alpha[tid] + (sm.red_sum[0][tid] + sm.red_sum[1][tid]) +
-                            (sm.red_sum[2][tid] + sm.red_sum[3][tid]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full);
-        }
-        if (!timed_out && nt > 0) {
-            const bool ok_wait = mbar_wait(&sm.o_done, (nt - 1) & 1);
-            timed_out = soft_sync_or(!ok_wait);
-        } else {
-            soft_sync();
-        }
-        if (!timed_out) {
-            tc_fence_after();
-            // ---- write O (normalised) or the split's partial (O, m, l)
-            const bool partial = splits > 1;
-            float* dst = partial ? ab.part_o + (int64_t)unit * H * D : P.out + (int64_t)b * H * D;
-            for (int c = hh * 2; c < hh * 2 + 2; ++c) {
-                const int lat = 128 * c + quad * 32 + lane;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float o[32];
-                    if (nt > 0) {
-                        tmem_ld_32x32b_x32(tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * c + 32 * half, o);
-                    } else {
-#pragma unroll
-                        for (int h = 0; h < 32; ++h) o[h] = 0.0f;
-                    }
-#pragma unroll
-                    for (int h = 0; h < 32; ++h) {
-                        const int hd = 32 * half + h;
-                        if (hd < H) {
-                            const float l = sm.l[hd];
-                            dst[(int64_t)hd * D + lat] = partial ? o[h] : (l > 0.0f ? o[h] / l : 0.0f);
+                            for (int k = 0; k < 4; ++k) {
+                                const uint32_t h = e2m1x2_to_h2((cw[c] >> (8 * k)) & 0xFFu);
+                                const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&h), s2);
+                                os[k] = *reinterpret_cast<const uint32_t*>(&v);
+                            }
+                            *reinterpret_cast<uint4*>(sm.items[j] + sw128(r, c)) = o;
                         }
                     }
                 }
             }
-            if (partial && tid < H) {
-                ab.part_ml[((int64_t)unit * H + tid) * 2 + 0] = sm.m_used[tid];
-                ab.part_ml[((int64_t)unit * H + tid) * 2 + 1] = sm.l[tid];
+        }
+        if (tid == 0) {
+            sm.n_entries[buf ^ 1] = 0;
+            sm.has_window[buf ^ 1] = 0;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(timed_out)) {
+            timed_out = true;
+            break;
+        }
+
+        // ---- S^T = Items . Q^T, and meanwhile the next tile's lookups
+        if (warp == 0) {
+            tc_fence_after();
+#pragma unroll 4
+            for (int ks = 0; ks < 32; ++ks) {  // 16 latent channels per MMA
+                const uint32_t off = (uint32_t)((ks >> 2) * (kT * 128) + (ks & 3) * 32) >> 4;
+                const uint32_t offq = (uint32_t)((ks >> 2) * (kHp * 128) + (ks & 3) * 32) >> 4;
+                tc_mma_f16_w(tbase + kColS, desc_items + off, desc_q + offq, idesc_s, ks > 0 ? 1u : 0u);
+            }
+            tc_commit_w(&sm.bar);
+        }
+        if (t + 1 < t_end) lookup(t + 1, buf ^ 1);
+        if (!mbar_wait(&sm.bar, phase)) timed_out = true;
+        phase ^= 1;
+        if (__syncthreads_or(timed_out)) {
+            timed_out = true;
+            break;
+        }
+        tc_fence_after();
+
+        // ---- softmax statistics: warp = (quadrant, head half); thread = item row
+        const int quad = warp & 3, hh = warp >> 2;
+        const int row = quad * 32 + lane;
+        const uint32_t s_addr = tbase + ((uint32_t)(quad * 32) << 16) + kColS + 32 * hh;
+        const bool ok = sm.kind[buf][row] != 0;
+        {
+            float v[32];
+            tmem_ld_32x32b_x32(s_addr, v);
+#pragma unroll
+            for (int h = 0; h < 32; ++h) v[h] = ok ? v[h] * ab.scale : -INFINITY;
+            warp_reduce_scatter<true, 32>(v);
+            sm.red[quad][32 * hh + lane] = v[0];
+        }
+        __syncthreads();
+        bool rescale = false;
+        if (tid < kHp) {
+            const float mt = fmaxf(fmaxf(sm.red[0][tid], sm.red[1][tid]), fmaxf(sm.red[2][tid], sm.red[3][tid]));
+            const float mo = sm.m_used[tid];
+            float a = 1.0f;
+            if (mt > mo + kRescaleGap || (mo == -INFINITY && mt != -INFINITY)) {
+                a = (mo == -INFINITY) ? 0.0f : expf(mo - mt);
+                sm.m_used[tid] = mt;
+                rescale = o_init && mo != -INFINITY;
+            }
+            sm.alpha[tid] = a;
+        }
+        rescale = __syncthreads_or(rescale);
+
+        // ---- P^T = exp(s - m) in fp16 (S reloaded from TMEM), row sums of the rounded p
+        {
+            float v[32];
+            tmem_ld_32x32b_x32(s_addr, v);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint4 o;
+                uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int h = 8 * c + 2 * k;
+                    const float p0 = ok ? __expf(v[h] * ab.scale - sm.m_used[32 * hh + h]) : 0.0f;
+                    const float p1 = ok ? __expf(v[h + 1] * ab.scale - sm.m_used[32 * hh + h + 1]) : 0.0f;
+                    const __half2 hv = __floats2half2_rn(p0, p1);
+                    const float2 back = __half22float2(hv);
+                    v[h] = back.x;
+                    v[h + 1] = back.y;
+                    os[k] = *reinterpret_cast<const uint32_t*>(&hv);
+                }
+                *reinterpret_cast<uint4*>(sm.p + sw128(row, 4 * hh + c)) = o;
+            }
+            warp_reduce_scatter<false, 32>(v);
+            // the max pass read red[] before the barrier above; reuse it for sums
+            sm.red[quad][32 * hh + lane] = v[0];
+        }
+        // ---- rescale O^T where a head's reference maximum moved
+        if (rescale) {
+            for (int c = hh * 2; c < hh * 2 + 2; ++c) {
+                const uint32_t ta = tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * c;
+                float o[64];
+                tmem_ld_32x32b_x64(ta, o);
+#pragma unroll
+                for (int h = 0; h < 64; ++h) o[h] *= sm.alpha[h];
+                tmem_st_32x32b_x64(ta, o);
             }
         }
-    }
-    if (timed_out && K > 0 && lane == 0) atomicOr(P.cache.status, CSA2_DEVERR_TIMEOUT);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid < kHp)
+            sm.l[tid] = sm.l[tid] * sm.alpha[tid] + (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
 
+        // ---- O^T += Items^T . P^T
+        if (warp == 0) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll 4
+                for (int i = 0; i < 8; ++i) {  // 16 items per MMA
+                    const uint32_t offa = (uint32_t)(2 * c * (kT * 128) + 2048 * i) >> 4;
+                    const uint32_t offp = (uint32_t)(2048 * i) >> 4;
+                    tc_mma_f16_w(tbase + kColO + 64 * c, desc_vt + offa, desc_p + offp, idesc_o,
+                                 (o_init || i > 0) ? 1u : 0u);
+                }
+            }
+            tc_commit_w(&sm.bar);
+        }
+        o_init = true;
+        if (t + 1 < t_end) load_entries(buf ^ 1);  // in flight while O runs
+        if (!mbar_wait(&sm.bar, phase)) timed_out = true;
+        phase ^= 1;
+        if (__syncthreads_or(timed_out)) {
+            timed_out = true;
+            break;
+        }
+        tc_fence_after();
+    }
+
+    if (timed_out) {
+        if (tid == 0 && K > 0) atomicOr(P.cache.status, CSA2_DEVERR_TIMEOUT);
+    } else {
+        // ---- write O (normalised) or the split's partial (O, m, l)
+        const int quad = warp & 3;
+        const bool partial = splits > 1;
+        float* dst = partial ? ab.part_o + (int64_t)unit * H * D : P.out + (int64_t)b * H * D;
+        for (int c = (warp >> 2) * 2; c < (warp >> 2) * 2 + 2; ++c) {
+            float o[64];
+            if (o_init) {
+                tmem_ld_32x32b_x64(tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * c, o);
+            } else {
+#pragma unroll
+                for (int h = 0; h < 64; ++h) o[h] = 0.0f;
+            }
+            const int lat = 128 * c + quad * 32 + lane;
+#pragma unroll
+            for (int h = 0; h < 64; ++h) {
+                if (h < H) {
+                    const float l = sm.l[h];
+                    dst[(int64_t)h * D + lat] = partial ? o[h] : (l > 0.0f ? o[h] / l : 0.0f);
+                }
+            }
+        }
+        if (partial && tid < H) {
+            ab.part_ml[((int64_t)unit * H + tid) * 2 + 0] = sm.m_used[tid];
+            ab.part_ml[((int64_t)unit * H + tid) * 2 + 1] = sm.l[tid];
+        }
+    }
+    // a timed-out wait may leave copies in flight: let them land before the CTA exits
+    if (tid == 0) {
+        (void)mbar_wait(&sm.wbar, wphase ^ 1);
+    }
     tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
     }
@@ -609,12 +532,7 @@ int attn_mma_splits(int n_problems, int batch, int Kmax) {
     return std::max(1, std::min(tiles, want));
 }
 
-bool attn_mma_supported(const AttnBatch& ab) {
-    if (ab.H < 1 || ab.H > kHp || ab.Kmax > CSA2_MAX_K) return false;
-    for (int i = 0; i < ab.n; ++i)  // entry rows are kept as 32-bit ints
-        if (ab.p[i].K > 0 && (int64_t)ab.p[i].cache.num_pages * PAGE > INT32_MAX) return false;
-    return true;
-}
+bool attn_mma_supported(const AttnBatch& ab) { return ab.H >= 1 && ab.H <= kHp; }
 
 size_t attn_mma_workspace_bytes(int n_problems, int batch, int H, int Kmax) {
     const int splits = attn_mma_splits(n_problems, batch, Kmax);
