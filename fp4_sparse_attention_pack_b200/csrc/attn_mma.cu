@@ -16,16 +16,15 @@
 // a tile's maximum exceeds it by more than 8 (so p <= e^8 fits fp16), which
 // makes the O rescale (TMEM load, scale, store) rare.  Heads are padded to 64.
 //
-// CTA = 256 threads, one unit (problem, sequence, split of tiles) per CTA.
+// CTA = 512 threads, one unit (problem, sequence, split of tiles) per CTA.
 // Gather: the unit's selected entries and window are prefetched into L2 first;
 // window rows arrive by TMA (a 3-D tensor map per window, 128-byte swizzle, one
 // box per slab, so they land directly in the slab layout and are converted
-// bf16 -> fp16 in place); cache entries are loaded with 16-byte loads (eight
-// lanes per entry row) and dequantised in registers, the chunk order staggered
-// per lane so the swizzled stores are free of bank conflicts.  Warp 0 issues the MMAs (one
-// elected lane, the warp converged); all eight
-// warps run the softmax (two per TMEM lane quadrant, 32 heads each) and
-// rescale / write O.
+// bf16 -> fp16 in place); cache entries are loaded with 16-byte loads into
+// registers one tile ahead (warp w: slab w % 8, rows 64 (w / 8) .. + 63, two rows
+// per lane) and dequantised into the swizzled slab.  Warp 0 issues the MMAs (one
+// elected lane, the warp converged); all sixteen warps run the softmax (four per
+// TMEM lane quadrant, 16 heads each) and rescale / write O (one O^T block each).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,7 +45,7 @@ using namespace sm100;
 
 constexpr int kT = 128;            // items per tile (MMA M of S^T)
 constexpr int kHp = 64;            // heads, padded (MMA N)
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S^T: 64 columns
 constexpr uint32_t kColO = 64;     // O^T: 4 x 64 columns
@@ -108,8 +107,9 @@ __device__ __forceinline__ void zero_row(uint8_t* slab, int r) {
     for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(slab + sw128(r, c)) = make_uint4(0, 0, 0, 0);
 }
 
-// Reduce-scatter over the warp: v[N] per lane (N = 32 or 64) -> lane l holds the
-// reduction over the 32 lanes of element N/32 * l + i in v[i], i < N/32.
+// Reduce-scatter over the warp: v[N] per lane (N = 16, 32 or 64).  For N >= 32
+// lane l ends with the reduction over the 32 lanes of element N/32 * l + i in
+// v[i], i < N/32; for N = 16 lanes 2e and 2e + 1 both hold element e in v[0].
 template <bool kMax, int N>
 __device__ __forceinline__ void warp_reduce_scatter(float (&v)[N]) {
     const int lane = threadIdx.x & 31;
@@ -117,13 +117,18 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&v)[N]) {
     for (int step = 0; step < 5; ++step) {
         const int o = 16 >> step;
         const int half = (N / 2) >> step;
-        const bool upper = (lane & o) != 0;
+        if (half >= 1) {
+            const bool upper = (lane & o) != 0;
 #pragma unroll
-        for (int i = 0; i < half; ++i) {
-            const float keep = upper ? v[half + i] : v[i];
-            const float send = upper ? v[i] : v[half + i];
-            const float got = __shfl_xor_sync(0xffffffffu, send, o);
-            v[i] = kMax ? fmaxf(keep, got) : keep + got;
+            for (int i = 0; i < half; ++i) {
+                const float keep = upper ? v[half + i] : v[i];
+                const float send = upper ? v[i] : v[half + i];
+                const float got = __shfl_xor_sync(0xffffffffu, send, o);
+                v[i] = kMax ? fmaxf(keep, got) : keep + got;
+            }
+        } else {
+            const float got = __shfl_xor_sync(0xffffffffu, v[0], o);
+            v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
         }
     }
 }
@@ -160,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.l[tid] = 0.0f;
     }
     // Q -> fp16 slabs (rows >= H are zero): cp.async in place, then convert.
-    {
+    if (warp < 8) {
         const int j = warp;
         for (int h = lane; h < kHp; h += 32) {
             if (h < H) {
@@ -239,14 +244,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     };
-    // Packed bytes of the tile's cache entries: warp = slab j, lane = rows lane + 32 i.
-    uint4 raw0[4], raw1[4];
-    uint32_t raws[4];
+    // Packed bytes of the tile's cache entries: warp w takes slab w & 7 of rows
+    // 64 (w >> 3) .. 64 (w >> 3) + 63, lane = rows lane + 32 i of that half.
+    const int g_slab = warp & 7, g_row0 = 64 * (warp >> 3);
+    uint4 raw0[2], raw1[2];
+    uint32_t raws[2];
     auto load_entries = [&](int buf) {
-        const int j = warp;
+        const int j = g_slab;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = lane + 32 * i;
+        for (int i = 0; i < 2; ++i) {
+            const int r = g_row0 + lane + 32 * i;
             if (sm.kind[buf][r] == 1) {
                 const int64_t ent = sm.src_row[buf][r];
                 const uint4* cs = reinterpret_cast<const uint4*>(P.cache.main_codes + ent * MCB + 32 * j);
@@ -275,17 +282,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 8; ++j) tma_load_3d_w(sm.items[j], &maps.win[prob], 64 * j, t * kT - K, b, &sm.wbar);
         }
-        // ---- cache entries (bytes already in registers): warp = slab, lane = row.
+        // ---- cache entries (bytes already in registers): warp = (slab, row half), lane = row.
         // The window boxes cover all 128 rows, so they must land first.
         if (has_window) {
             if (!mbar_wait(&sm.wbar, wphase)) timed_out = true;
             wphase ^= 1;
         }
         {
-            const int j = warp;
+            const int j = g_slab;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = lane + 32 * i;
+            for (int i = 0; i < 2; ++i) {
+                const int r = g_row0 + lane + 32 * i;
                 const int kind = sm.kind[buf][r];
                 if (kind == 2) {
                     bf16_row_to_f16(sm.items[j], r);
@@ -345,18 +352,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
 
-        // ---- softmax statistics: warp = (quadrant, head half); thread = item row
-        const int quad = warp & 3, hh = warp >> 2;
+        // ---- softmax statistics: warp = (quadrant, 16 heads); thread = item row
+        const int quad = warp & 3, hq = warp >> 2;
         const int row = quad * 32 + lane;
-        const uint32_t s_addr = tbase + ((uint32_t)(quad * 32) << 16) + kColS + 32 * hh;
+        const uint32_t s_addr = tbase + ((uint32_t)(quad * 32) << 16) + kColS + 16 * hq;
         const bool ok = sm.kind[buf][row] != 0;
         {
-            float v[32];
-            tmem_ld_32x32b_x32(s_addr, v);
+            float v[16];
+            tmem_ld_32x32b_x16(s_addr, v);
 #pragma unroll
-            for (int h = 0; h < 32; ++h) v[h] = ok ? v[h] * ab.scale : -INFINITY;
-            warp_reduce_scatter<true, 32>(v);
-            sm.red[quad][32 * hh + lane] = v[0];
+            for (int h = 0; h < 16; ++h) v[h] = ok ? v[h] * ab.scale : -INFINITY;
+            warp_reduce_scatter<true, 16>(v);
+            if ((lane & 1) == 0) sm.red[quad][16 * hq + (lane >> 1)] = v[0];
         }
         __syncthreads();
         bool rescale = false;
@@ -375,38 +382,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // ---- P^T = exp(s - m) in fp16 (S reloaded from TMEM), row sums of the rounded p
         {
-            float v[32];
-            tmem_ld_32x32b_x32(s_addr, v);
+            float v[16];
+            tmem_ld_32x32b_x16(s_addr, v);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint4 o;
                 uint32_t* os = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int h = 8 * c + 2 * k;
-                    const float p0 = ok ? __expf(v[h] * ab.scale - sm.m_used[32 * hh + h]) : 0.0f;
-                    const float p1 = ok ? __expf(v[h + 1] * ab.scale - sm.m_used[32 * hh + h + 1]) : 0.0f;
+                    const float p0 = ok ? __expf(v[h] * ab.scale - sm.m_used[16 * hq + h]) : 0.0f;
+                    const float p1 = ok ? __expf(v[h + 1] * ab.scale - sm.m_used[16 * hq + h + 1]) : 0.0f;
                     const __half2 hv = __floats2half2_rn(p0, p1);
                     const float2 back = __half22float2(hv);
                     v[h] = back.x;
                     v[h + 1] = back.y;
                     os[k] = *reinterpret_cast<const uint32_t*>(&hv);
                 }
-                *reinterpret_cast<uint4*>(sm.p + sw128(row, 4 * hh + c)) = o;
+                *reinterpret_cast<uint4*>(sm.p + sw128(row, 2 * hq + c)) = o;
             }
-            warp_reduce_scatter<false, 32>(v);
+            warp_reduce_scatter<false, 16>(v);
             // the max pass read red[] before the barrier above; reuse it for sums
-            sm.red[quad][32 * hh + lane] = v[0];
+            if ((lane & 1) == 0) sm.red[quad][16 * hq + (lane >> 1)] = v[0];
         }
-        // ---- rescale O^T where a head's reference maximum moved
+        // ---- rescale O^T where a head's reference maximum moved (warp = quadrant, block hq)
         if (rescale) {
-            for (int c = hh * 2; c < hh * 2 + 2; ++c) {
-                const uint32_t ta = tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * c;
-                float o[64];
-                tmem_ld_32x32b_x64(ta, o);
+            const uint32_t ta = tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * hq;
 #pragma unroll
-                for (int h = 0; h < 64; ++h) o[h] *= sm.alpha[h];
-                tmem_st_32x32b_x64(ta, o);
+            for (int half = 0; half < 2; ++half) {
+                float o[32];
+                tmem_ld_32x32b_x32(ta + 32 * half, o);
+#pragma unroll
+                for (int h = 0; h < 32; ++h) o[h] *= sm.alpha[32 * half + h];
+                tmem_st_32x32b_x32(ta + 32 * half, o);
             }
         }
         fence_proxy_async_smem();
@@ -448,20 +456,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;
         const bool partial = splits > 1;
         float* dst = partial ? ab.part_o + (int64_t)unit * H * D : P.out + (int64_t)b * H * D;
-        for (int c = (warp >> 2) * 2; c < (warp >> 2) * 2 + 2; ++c) {
-            float o[64];
-            if (o_init) {
-                tmem_ld_32x32b_x64(tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * c, o);
-            } else {
-#pragma unroll
-                for (int h = 0; h < 64; ++h) o[h] = 0.0f;
-            }
+        {
+            const int c = warp >> 2;  // O^T block of this warp: latent 128 c + quad * 32 + lane
             const int lat = 128 * c + quad * 32 + lane;
 #pragma unroll
-            for (int h = 0; h < 64; ++h) {
-                if (h < H) {
-                    const float l = sm.l[h];
-                    dst[(int64_t)h * D + lat] = partial ? o[h] : (l > 0.0f ? o[h] / l : 0.0f);
+            for (int half = 0; half < 2; ++half) {
+                float o[32];
+                if (o_init) {
+                    tmem_ld_32x32b_x32(tbase + ((uint32_t)(quad * 32) << 16) + kColO + 64 * c + 32 * half, o);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) o[h] = 0.0f;
+                }
+#pragma unroll
+                for (int h = 0; h < 32; ++h) {
+                    const int hd = 32 * half + h;
+                    if (hd < H) {
+                        const float l = sm.l[hd];
+                        dst[(int64_t)hd * D + lat] = partial ? o[h] : (l > 0.0f ? o[h] / l : 0.0f);
+                    }
                 }
             }
         }
