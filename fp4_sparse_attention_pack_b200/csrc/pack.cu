@@ -64,6 +64,36 @@ __device__ __forceinline__ void stage_w(float* wb, const float* W, int k) {
     cp_async_commit();
 }
 
+// k[jj][o] for jj < ne <= NE: fma over c = 0..511 in order (thread o = threadIdx.x).
+template <int NE>
+__device__ __forceinline__ void project(float (&acc)[kEnt], const float* deq, float* wbuf, const float* W, int ne) {
+#pragma unroll
+    for (int jj = 0; jj < kEnt; ++jj) acc[jj] = 0.0f;
+    const int o = threadIdx.x;
+    constexpr int kSteps = D / kWc;
+    stage_w(wbuf, W, 0);
+#pragma unroll 1
+    for (int k = 0; k < kSteps; ++k) {
+        if (k + 1 < kSteps) {
+            stage_w(wbuf + ((k + 1) & 1) * kWc * DI, W, k + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const float* wb = wbuf + (k & 1) * kWc * DI;
+#pragma unroll 4
+        for (int cc = 0; cc < kWc; ++cc) {
+            const float w = wb[cc * DI + o];
+            const int ch = k * kWc + cc;
+#pragma unroll
+            for (int jj = 0; jj < NE; ++jj)
+                if (jj < ne) acc[jj] = __fmaf_rn(w, deq[jj * D + ch], acc[jj]);
+        }
+        __syncthreads();
+    }
+}
+
 template <bool kF32>
 __global__ void __launch_bounds__(kThreads) k_pack_entries(const __grid_constant__ PackBatch pb, int T) {
     extern __shared__ float deq[];  // [kEnt][512], then W staging [2][kWc][128]
@@ -138,35 +168,17 @@ __global__ void __launch_bounds__(kThreads) k_pack_entries(const __grid_constant
     __syncthreads();
 
     // ---- phase 2: k[jj][o] = sum_c W[c][o] * deq[jj][c], fma order c = 0..511,
-    // W rows staged through shared memory (double-buffered cp.async)
+    // W rows staged through shared memory (double-buffered cp.async).  A CTA with
+    // at most 4 entries (decode: one token per step) keeps 4 accumulators instead
+    // of kEnt, so it does not issue kEnt predicated FMAs per channel.
     float acc[kEnt];
-#pragma unroll
-    for (int jj = 0; jj < kEnt; ++jj) acc[jj] = 0.0f;
-    const int o = t;
-    constexpr int kSteps = D / kWc;
-    stage_w(wbuf, W, 0);
-#pragma unroll 1
-    for (int k = 0; k < kSteps; ++k) {
-        if (k + 1 < kSteps) {
-            stage_w(wbuf + ((k + 1) & 1) * kWc * DI, W, k + 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const float* wb = wbuf + (k & 1) * kWc * DI;
-#pragma unroll 4
-        for (int cc = 0; cc < kWc; ++cc) {
-            const float w = wb[cc * DI + o];
-            const int ch = k * kWc + cc;
-#pragma unroll
-            for (int jj = 0; jj < kEnt; ++jj)
-                if (jj < ne) acc[jj] = __fmaf_rn(w, deq[jj * D + ch], acc[jj]);
-        }
-        __syncthreads();
-    }
+    if (ne <= 4)
+        project<4>(acc, deq, wbuf, W, ne);
+    else
+        project<kEnt>(acc, deq, wbuf, W, ne);
 
     // ---- phase 3: MXFP4 per 32 channels (warp w = block w)
+    const int o = t;
     const int lane = t & 31, blk = t >> 5;
 #pragma unroll
     for (int jj = 0; jj < kEnt; ++jj) {

@@ -3,7 +3,7 @@
 // Scores map to order-preserving uint32 keys; the K largest are kept, equal
 // scores lower index first, and written in increasing index order.
 //
-// One CTA of 512 threads per (problem, sequence), four CTAs per SM:
+// One CTA of 512 threads per (problem, sequence):
 //   1. Threshold guess: 2,048 strided samples of the row; an exact radix select
 //      in shared memory finds the sample key ranked ~2K * 2048 / n, so that
 //      about 2K of the n scores lie at or above it.
@@ -161,7 +161,7 @@ __device__ void emit_topk(KeyAt key_at, IdxAt idx_at, int cnt, uint32_t kth, int
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 4) k_topk(const __grid_constant__ ScanBatch sb) {
+__global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanBatch sb) {
     extern __shared__ uint8_t smem_raw[];
     TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
     const ScanProblem& P = sb.p[blockIdx.y];

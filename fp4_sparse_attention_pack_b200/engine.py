@@ -109,25 +109,50 @@ class DecodeModel:
                                 self._w, self._wins, B, wl.H, wl.H_idx, wl.K, wl.scale)
         self.ws = torch.empty(max(layer_step_workspace(self.model), 16), dtype=torch.uint8, device=device)
         # per-step buffers
-        self.x_new = torch.zeros(self.S, B, D, dtype=torch.bfloat16, device=device)
-        self.g_new = torch.zeros(self.S, B, dtype=torch.float32, device=device)
-        self.q = torch.zeros(self.L, B, wl.H, D, dtype=torch.bfloat16, device=device)
-        self.q_idx = torch.zeros(self.L, B, wl.H_idx, D_IDX, dtype=torch.bfloat16, device=device)
-        self.w = torch.zeros(self.L, B, wl.H_idx, dtype=torch.float32, device=device)
-        self.win_tok = torch.zeros(self.L, B, D, dtype=torch.bfloat16, device=device)
-        self.out = torch.zeros(self.L, B, wl.H, D, dtype=torch.float32, device=device)
-        self.idx = torch.full((self.L, B, wl.K), -1, dtype=torch.int32, device=device)
-        scan = set(t.scan_layers())
-        self._in = csa2_step_in(
-            _ptr_array([self.x_new[s] for s in range(self.S)]),
-            _ptr_array([self.g_new[s] for s in range(self.S)]),
-            _ptr_array([self.q[l] for l in range(self.L)]),
-            _ptr_array([self.q_idx[l] if l in scan else None for l in range(self.L)]),
-            _ptr_array([self.w[l] if l in scan else None for l in range(self.L)]),
-            _ptr_array([self.win_tok[l] for l in range(self.L)]))
-        self._out = csa2_step_out(_ptr_array([self.out[l] for l in range(self.L)]),
-                                  _ptr_array([self.idx[l] if l in scan else None for l in range(self.L)]))
+        self.io = self.new_io()
+        (self.x_new, self.g_new, self.q, self.q_idx, self.w, self.win_tok, self.out,
+         self.idx) = self.io.tensors
+        self._in, self._out = self.io.step_in, self.io.step_out
         self.position = wl.T  # tokens already in every stream
+
+    class IO:
+        """One set of per-step device buffers and the C structs that point at them."""
+
+        def __init__(self, tensors, step_in, step_out, keep):
+            self.tensors, self.step_in, self.step_out, self._keep = tensors, step_in, step_out, keep
+
+        @property
+        def inputs(self):
+            return list(self.tensors[:6])
+
+        @property
+        def outputs(self):
+            return list(self.tensors[6:])
+
+    def new_io(self) -> "DecodeModel.IO":
+        """A fresh set of step inputs (x_new, g_new, q, q_idx, w, win_tok) and outputs
+        (out, idx); several sets let copies of one step overlap the compute of another."""
+        wl, B, dev = self.wl, self.wl.B, self.dev
+        x_new = torch.zeros(self.S, B, D, dtype=torch.bfloat16, device=dev)
+        g_new = torch.zeros(self.S, B, dtype=torch.float32, device=dev)
+        q = torch.zeros(self.L, B, wl.H, D, dtype=torch.bfloat16, device=dev)
+        q_idx = torch.zeros(self.L, B, wl.H_idx, D_IDX, dtype=torch.bfloat16, device=dev)
+        w = torch.zeros(self.L, B, wl.H_idx, dtype=torch.float32, device=dev)
+        win_tok = torch.zeros(self.L, B, D, dtype=torch.bfloat16, device=dev)
+        out = torch.zeros(self.L, B, wl.H, D, dtype=torch.float32, device=dev)
+        idx = torch.full((self.L, B, wl.K), -1, dtype=torch.int32, device=dev)
+        scan = set(self.wl.table.scan_layers())
+        arrays = [_ptr_array([x_new[s] for s in range(self.S)]),
+                  _ptr_array([g_new[s] for s in range(self.S)]),
+                  _ptr_array([q[l] for l in range(self.L)]),
+                  _ptr_array([q_idx[l] if l in scan else None for l in range(self.L)]),
+                  _ptr_array([w[l] if l in scan else None for l in range(self.L)]),
+                  _ptr_array([win_tok[l] for l in range(self.L)])]
+        outs = [_ptr_array([out[l] for l in range(self.L)]),
+                _ptr_array([idx[l] if l in scan else None for l in range(self.L)])]
+        step_in = csa2_step_in(*arrays)
+        step_out = csa2_step_out(*outs)
+        return DecodeModel.IO((x_new, g_new, q, q_idx, w, win_tok, out, idx), step_in, step_out, arrays + outs)
 
     # ---------------------------------------------------------------- filling
     def fill(self, chunk_tokens: int = 8192):
@@ -197,8 +222,9 @@ class DecodeModel:
             synth.dev_normal_bf16_rows(self.win_tok[l], synth.key(wl.seed, synth.TID_WIN, l), p * D,
                                        synth.TSTRIDE * D, B, D)
 
-    def step(self, stream=None):
-        layer_step(self.model, self._in, self._out, self.ws, stream)
+    def step(self, stream=None, io=None):
+        io = self.io if io is None else io
+        layer_step(self.model, io.step_in, io.step_out, self.ws, stream)
 
     def status_bits(self) -> int:
         return max(c.status_bits() for c in self.caches)
