@@ -22,7 +22,9 @@
 // box per slab, so they land directly in the slab layout and are converted
 // bf16 -> fp16 in place); cache entries are loaded with 16-byte loads into
 // registers one tile ahead (warp w: slab w % 8, rows 64 (w / 8) .. + 63, two rows
-// per lane) and dequantised into the swizzled slab.  Warp 0 issues the MMAs (one
+// per lane) and dequantised into the swizzled slab; a slab is rewritten as soon
+// as the previous tile's O block that reads it has completed (the O MMAs commit
+// per 128-channel block), so the gather overlaps O.  Warp 0 issues the MMAs (one
 // elected lane, the warp converged); all sixteen warps run the softmax (four per
 // TMEM lane quadrant, 16 heads each) and rescale / write O (one O^T block each).
 #include <cuda.h>
@@ -67,8 +69,10 @@ struct __align__(1024) Smem {
     int64_t src_row[2][kT];        // entry row in the pools
     int n_entries[2];
     int has_window[2];
-    uint64_t bar;                  // MMA completion
+    uint64_t bar;                  // S MMA completion
+    uint64_t ob[4];                // O MMA completion per 128-channel block (slabs 2c, 2c + 1)
     uint64_t wbar;                 // window TMA
+    uint64_t drained;              // every MMA of the unit completed
     uint32_t tmem_base;
 };
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory beyond the 227 KB per-block limit");
@@ -153,7 +157,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         mbar_init(&sm.bar, 1);
+        for (int c = 0; c < 4; ++c) mbar_init(&sm.ob[c], 1);
         mbar_init(&sm.wbar, 1);
+        mbar_init(&sm.drained, 1);
         sm.n_entries[0] = sm.n_entries[1] = 0;
         sm.has_window[0] = sm.has_window[1] = 0;
         fence_mbar_init();
@@ -275,9 +281,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = t_begin; t < t_end && !timed_out; ++t, buf ^= 1) {
         const bool has_window = sm.has_window[buf] != 0;
-        // ---- window rows by TMA, one 64-channel box per slab (O of the previous
-        // tile has completed, so the item buffer is free)
+        // The O MMAs of the previous tile read slabs 2c, 2c + 1 in block c; a slab is
+        // rewritten once its block has completed (phase of the previous tile's O).
+        const uint32_t opar = (uint32_t)(t - t_begin - 1) & 1u;
+        // ---- window rows by TMA, one 64-channel box per slab, once every block of
+        // the previous tile's O has completed (the last block's commit covers all)
         if (warp == 0 && has_window) {
+            if (o_init && !mbar_wait_warp(&sm.ob[3], opar)) timed_out = true;
             mbar_expect_tx_w(&sm.wbar, 8 * kT * 128);
 #pragma unroll
             for (int j = 0; j < 8; ++j) tma_load_3d_w(sm.items[j], &maps.win[prob], 64 * j, t * kT - K, b, &sm.wbar);
@@ -287,6 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (has_window) {
             if (!mbar_wait(&sm.wbar, wphase)) timed_out = true;
             wphase ^= 1;
+        } else if (o_init) {
+            if (!mbar_wait(&sm.ob[g_slab >> 1], opar)) timed_out = true;
         }
         {
             const int j = g_slab;
@@ -435,13 +447,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_mma_f16_w(tbase + kColO + 64 * c, desc_vt + offa, desc_p + offp, idesc_o,
                                  (o_init || i > 0) ? 1u : 0u);
                 }
+                tc_commit_w(&sm.ob[c]);
             }
-            tc_commit_w(&sm.bar);
         }
         o_init = true;
-        if (t + 1 < t_end) load_entries(buf ^ 1);  // in flight while O runs
-        if (!mbar_wait(&sm.bar, phase)) timed_out = true;
-        phase ^= 1;
+        // the next tile's gather overlaps these MMAs, slab pair by slab pair
+        if (t + 1 < t_end) load_entries(buf ^ 1);
         if (__syncthreads_or(timed_out)) {
             timed_out = true;
             break;
@@ -449,6 +460,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
     }
 
+    // the last tile's O has completed before it is read (its last block covers all)
+    if (!timed_out && o_init) {
+        const bool ok = mbar_wait(&sm.ob[3], (uint32_t)(t_end - t_begin - 1) & 1u);
+        timed_out = __syncthreads_or(!ok);
+        tc_fence_after();
+    }
     if (timed_out) {
         if (tid == 0 && K > 0) atomicOr(P.cache.status, CSA2_DEVERR_TIMEOUT);
     } else {
@@ -486,6 +503,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a timed-out wait may leave copies in flight: let them land before the CTA exits
     if (tid == 0) {
         (void)mbar_wait(&sm.wbar, wphase ^ 1);
+    }
+    // every MMA of warp 0 has completed before TMEM is freed
+    if (warp == 0) {
+        tc_commit_w(&sm.drained);
+        (void)mbar_wait_warp(&sm.drained, 0);
     }
     tc_fence_before();
     __syncthreads();
