@@ -14,12 +14,13 @@ from ._build import LIB
 
 __all__ = ["Csa2Error", "lib", "csa2_cache", "csa2_window", "csa2_model", "csa2_step_in",
            "csa2_step_out", "pack_cache", "index_topk", "index_topk_workspace", "sparse_attn",
-           "sparse_attn_workspace", "window_append", "layer_step", "layer_step_workspace", "layer_step_launches",
+           "sparse_attn_workspace", "window_append", "layer_step", "layer_step_workspace", "layer_step_launches", "seq_image_bytes", "cache_export",
+           "cache_import",
            "SWA_ONLY", "FULL", "REINDEX", "REUSE", "DTYPE_BF16", "DTYPE_F32"]
 
 SWA_ONLY, FULL, REINDEX, REUSE = 0, 1, 2, 3
 DTYPE_BF16, DTYPE_F32 = 0, 1
-DEVERR_CAPACITY, DEVERR_PAGE, DEVERR_COUNT, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_CAPACITY, DEVERR_PAGE, DEVERR_COUNT, DEVERR_TIMEOUT, DEVERR_IMAGE = 1, 2, 4, 8, 16
 
 _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
 
@@ -85,6 +86,9 @@ def lib():
             ("csa2_layer_step", ctypes.c_int, [P(csa2_model), P(csa2_step_in), P(csa2_step_out), _vp,
                                                _sz, _vp]),
             ("csa2_layer_step_launches", ctypes.c_int, [P(csa2_model), P(csa2_step_in)]),
+            ("csa2_seq_image_bytes", _sz, [ctypes.c_int]),
+            ("csa2_cache_export", ctypes.c_int, [P(csa2_cache), ctypes.c_int, _vp, ctypes.c_int, _vp]),
+            ("csa2_cache_import", ctypes.c_int, [P(csa2_cache), ctypes.c_int, _vp, ctypes.c_int, _vp]),
         ]:
             f = getattr(L, name)
             f.restype = res
@@ -160,6 +164,24 @@ def layer_step_launches(model: csa2_model, step_in: csa2_step_in) -> int:
     if n < 0:
         raise Csa2Error(n, "csa2_layer_step_launches")
     return n
+
+
+def seq_image_bytes(capacity: int) -> int:
+    """Bytes of a one-sequence cache image with room for `capacity` entries."""
+    return int(lib().csa2_seq_image_bytes(capacity))
+
+
+def cache_export(cache: csa2_cache, seq: int, image, capacity: int, stream=None):
+    """Copy sequence `seq` of `cache` into `image` (a uint8 tensor the device can
+    address: CUDA memory or pinned host memory) in logical entry order."""
+    _ok(lib().csa2_cache_export(ctypes.byref(cache), seq, _ptr(image), capacity, _stream(stream)),
+        "csa2_cache_export")
+
+
+def cache_import(cache: csa2_cache, seq: int, image, capacity: int, stream=None):
+    """Write an image made by cache_export into sequence `seq` of `cache`."""
+    _ok(lib().csa2_cache_import(ctypes.byref(cache), seq, _ptr(image), capacity, _stream(stream)),
+        "csa2_cache_import")
 
 
 def index_topk_noalloc(cache: csa2_cache, q_idx, w, K: int, idx_out, score_out=None, stream=None):

@@ -91,6 +91,7 @@ typedef enum { CSA2_DTYPE_BF16 = 0, CSA2_DTYPE_F32 = 1 } csa2_dtype;
 #define CSA2_DEVERR_PAGE 0x2u     /* a page-table entry is outside [0, num_pages) */
 #define CSA2_DEVERR_COUNT 0x4u    /* n_entries outside [0, max_pages * 64] */
 #define CSA2_DEVERR_TIMEOUT 0x8u  /* a bounded device wait gave up */
+#define CSA2_DEVERR_IMAGE 0x10u   /* a sequence image's header does not fit the cache (see import) */
 
 /*
  * One source layer's compressed cache for `batch` sequences, paged.
@@ -312,6 +313,44 @@ int csa2_index_topk_noalloc(const csa2_cache* cache, const uint16_t* q_idx, cons
 int csa2_layer_step_profiled(const csa2_model* model, const csa2_step_in* in,
                              const csa2_step_out* out, void* ws, size_t ws_bytes,
                              csa2_stream stream, void* const* events);
+
+/*
+ * Prefix-cache export / import of one sequence ("DeepSeek-V4.1-Flash,
+ * expliqué pas à pas": the introduction names the prefix cache, a session's
+ * cache reloaded instead of recomputed; the FP4-cache section keeps the global
+ * cache whole in the persistent store).  The pages give the feature, not a
+ * format; this image format is this library's own.
+ *
+ * A sequence image with room for `capacity` entries is, in order:
+ *   header   int32 n_entries, int32 pend_valid, float pend_g, int32 ratio (16 B)
+ *   pend_x   fp32[512]
+ *   main_codes [capacity][256], main_scales [capacity][32],
+ *   idx_codes  [capacity][64],  idx_scales  [capacity][4]
+ * with entries in logical order (entry e of the sequence at row e), the byte
+ * layout of each row as in csa2_cache.  csa2_seq_image_bytes(capacity) is its
+ * size: 2,064 + 356 * capacity bytes.
+ *
+ * csa2_cache_export copies sequence `seq` of `cache` into `image`: the header,
+ * the pending slot and the first n = n_entries[seq] rows; when n > capacity only
+ * `capacity` rows are copied, the header records that many, and
+ * CSA2_DEVERR_CAPACITY is set.  csa2_cache_import writes an image back into
+ * sequence `seq` of a cache (any page table, same ratio): its n rows go to the
+ * pages the page table gives, and n_entries and the pending slot are set.  An
+ * image whose ratio differs from the cache's, or whose n is negative or larger
+ * than min(capacity, max_pages * 64), is not imported (nothing written) and
+ * CSA2_DEVERR_IMAGE is set.  Rows whose page id is outside the pool are skipped
+ * with CSA2_DEVERR_PAGE.
+ *
+ * `image` is caller-owned memory the device can address (device memory, or
+ * pinned host memory mapped into the device address space), 16-byte aligned.
+ * Both calls are asynchronous on `stream`, read n_entries and the header on the
+ * device (no host synchronisation) and may be captured in a CUDA graph.
+ * Returns CSA2_ERR_INVALID_ARG for a NULL pointer, seq outside [0, batch) or
+ * capacity < 0; CSA2_ERR_ALIGN for an unaligned image.
+ */
+size_t csa2_seq_image_bytes(int capacity);
+int csa2_cache_export(const csa2_cache* cache, int seq, void* image, int capacity, csa2_stream stream);
+int csa2_cache_import(const csa2_cache* cache, int seq, const void* image, int capacity, csa2_stream stream);
 
 /*
  * Number of kernel launches one csa2_layer_step(model, in, ...) call enqueues

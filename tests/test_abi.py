@@ -71,6 +71,24 @@ def test_argument_checks_fail_before_launch(capi):
     assert capi.sparse_attn_workspace(2, 64, 512) > 0
 
 
+def test_cache_io_argument_checks(capi):
+    lib = capi.lib()
+    assert capi.seq_image_bytes(0) == 16 + 2048
+    assert capi.seq_image_bytes(10) == 16 + 2048 + 10 * (256 + 32 + 64 + 4)
+    assert lib.csa2_seq_image_bytes(-1) == 0
+    c = capi.csa2_cache(*([16] * 10), 2, 1, 1, 2)
+    img = ctypes.c_void_p(32)
+    for f in (lib.csa2_cache_export, lib.csa2_cache_import):
+        assert f(None, 0, img, 4, None) == -1                       # no cache
+        assert f(ctypes.byref(c), 0, None, 4, None) == -1           # no image
+        assert f(ctypes.byref(c), 2, img, 4, None) == -1            # seq outside [0, batch)
+        assert f(ctypes.byref(c), -1, img, 4, None) == -1
+        assert f(ctypes.byref(c), 0, img, -1, None) == -1           # negative capacity
+        assert f(ctypes.byref(c), 0, ctypes.c_void_p(40), 4, None) == -2  # unaligned image
+    c_bad = capi.csa2_cache(*([16] * 10), 2, 1, 1, 3)
+    assert lib.csa2_cache_export(ctypes.byref(c_bad), 0, img, 4, None) == -1  # bad ratio
+
+
 def test_mode_table_validation(capi):
     import numpy as np
     from fp4_sparse_attention_pack_b200 import workloads as W
