@@ -213,9 +213,11 @@ def oracle_sample(wl, seqs=(0,), layers=None, budget_s=None):
             oracle.attention(W.query(wl, l, 0)[b], items, wl.scale)
             dt = time.perf_counter() - t0
             (t_scan if m in (W.FULL, W.REINDEX) else t_attn).append(dt)
-    desc = (f"oracle on layers {layers[0]}-{layers[-1]} x sequences {list(seqs)} of the 40-layer "
-            f"step (Top-K scan over {wl.T // 2} entries, 64 heads, attention over K + 128 items); "
-            f"per-layer-step time = 16 x (23 scan-layer + 17 attention-only-layer) sequence times")
+    n_scan = len(t.scan_layers())
+    desc = (f"oracle on layers {layers[0]}-{layers[-1]} x sequences {list(seqs)} of the {t.n_layers}-layer "
+            f"step (Top-K scan over {wl.T // t.ratios[t.src[layers[0]]]} entries, {wl.H_idx} heads, attention "
+            f"over K + 128 items); per-layer-step time = {wl.B} x ({n_scan} scan-layer + "
+            f"{t.n_layers - n_scan} attention-only-layer) sequence times")
     return (statistics.mean(t_scan) if t_scan else 0.0, statistics.mean(t_attn) if t_attn else 0.0,
             oracle.threads(), desc)
 

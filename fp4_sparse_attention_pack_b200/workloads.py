@@ -131,6 +131,8 @@ WORKLOADS = {
                 outliers=True),
     4: Workload("cfg4_prefix_append_b16_256k", 4, 16, 262144, schedule_alternating_40(), 64, 64, 512,
                 64, append=8192),
+    # the pages' own schedule and ratios (8 scans per step, decoder source at ratio 1)
+    5: Workload("cfg5_pages40_b16_128k", 5, 16, 131072, schedule_pages_40(), 64, 64, 512, 100),
 }
 
 
