@@ -192,6 +192,49 @@ def topk(scores, K) -> np.ndarray:
     return out
 
 
+# Hierarchical sparse indexer ("DeepSeek-V4.1-Flash, expliqué pas à pas", CSA2
+# chapter, hierarchical indexer paragraph: in the CED decoder the shallow
+# indexer's information restricts the candidates of the deeper indexers, so only
+# the first Full layer keeps scanning the whole context; the video-summary page
+# gives the pool as blocks of 8 positions, 2,048 of them at a million tokens,
+# built by the first decoder layer).  The step list itself did not survive on
+# the page; the reading taken here: a block is 8 consecutive entries, its score
+# the largest score of its entries under the Full layer's indexer; the pool is
+# the pool_blocks best blocks (ties: lower block); a deeper Reindex layer scores
+# only the pool's entries and keeps its Top-K among them.
+POOL_BLOCK = 8
+
+
+def block_pool(scores, pool_blocks: int) -> np.ndarray:
+    """Block ids of the pool, increasing, padded with -1 (int32[pool_blocks])."""
+    scores = np.asarray(scores, np.float64)
+    n = scores.size
+    if n == 0:
+        return np.full(pool_blocks, -1, np.int32)
+    starts = np.arange(0, n, POOL_BLOCK)
+    bmax = np.maximum.reduceat(scores, starts)
+    return topk(bmax, pool_blocks)
+
+
+def pool_entries(pool, n: int) -> np.ndarray:
+    """Entries of the pool's blocks below n, increasing (int64)."""
+    blocks = np.asarray(pool, np.int64)
+    blocks = blocks[blocks >= 0]
+    ents = np.sort((blocks[:, None] * POOL_BLOCK + np.arange(POOL_BLOCK)[None, :]).reshape(-1))
+    return ents[ents < n]
+
+
+def topk_in_pool(scores, pool, K: int) -> np.ndarray:
+    """Top-K over the pool's entries only (score desc, entry asc), increasing,
+    padded with -1 (int32[K])."""
+    scores = np.asarray(scores, np.float64)
+    ents = pool_entries(pool, scores.size)
+    sel = topk(scores[ents], K)
+    if ents.size == 0:
+        return sel
+    return np.where(sel >= 0, ents[np.maximum(sel, 0)], -1).astype(np.int32)
+
+
 def attention_items(mc, ms, n_entries, idx, win_bf16, win_len) -> np.ndarray:
     idx = np.ascontiguousarray(idx, np.int32)
     win = np.ascontiguousarray(win_bf16, np.uint16)
@@ -248,9 +291,11 @@ class RefCache:
 class RefModel:
     """All layers of one decode model: per-source caches and per-layer windows."""
 
-    def __init__(self, table, B: int, caps, Ws, H: int, H_idx: int, K: int, scale: float):
+    def __init__(self, table, B: int, caps, Ws, H: int, H_idx: int, K: int, scale: float,
+                 pool_blocks: int = 0):
         self.t = table
         self.B, self.H, self.H_idx, self.K, self.scale = B, H, H_idx, K, scale
+        self.pool_blocks = pool_blocks  # > 0: Reindex layers search the Full layer's pool
         self.caches = [RefCache(B, caps[s], table.ratios[s], Ws[s]) for s in range(table.n_sources)]
         L = table.n_layers
         self.win = np.zeros((L, B, WIN, D), np.uint16)
@@ -296,12 +341,20 @@ class RefModel:
                 self.caches[s].append(b, x_new[s][b], g_new[s][b:b + 1])
         idx = [[None] * B for _ in range(L)]
         out = [[None] * B for _ in range(L)]
+        self.pools = {}  # (source, seq) -> pool of the source's Full layer this step
         for l in range(L):
             m = self.t.mode[l]
             for b in range(B):
                 if m in (FULL, REINDEX):
                     c = self.caches[self.t.src[l]]
-                    idx[l][b] = topk(c.scores(b, qidx[l][b], wh[l][b]), self.K)
+                    sc = c.scores(b, qidx[l][b], wh[l][b])
+                    pool = self.pools.get((self.t.src[l], b)) if self.pool_blocks > 0 else None
+                    if m == REINDEX and pool is not None:
+                        idx[l][b] = topk_in_pool(sc, pool, self.K)
+                    else:
+                        idx[l][b] = topk(sc, self.K)
+                    if m == FULL and self.pool_blocks > 0:
+                        self.pools[(self.t.src[l], b)] = block_pool(sc, self.pool_blocks)
                 elif m == REUSE:
                     idx[l][b] = idx[self.t.idx_src[l]][b]
                 if want is None or (l, b) in want:
