@@ -140,10 +140,13 @@ def kernel_traffic(kernel: str):
 
 def workload_config(wl, world):
     """The workload keys of the JSON line's config (both arms)."""
-    return {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.T,
-            "layers": wl.table.n_layers, "scans_per_step": len(wl.table.scan_layers()), "H": wl.H,
-            "H_idx": wl.H_idx, "top_k": wl.K, "parallelism": f"dp{world} (replicas, no collective)",
-            "cache_format": "E2M1+E4M3/16 main, MXFP4 indexer keys"}
+    cfg = {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.T,
+           "layers": wl.table.n_layers, "scans_per_step": len(wl.table.scan_layers()), "H": wl.H,
+           "H_idx": wl.H_idx, "top_k": wl.K, "parallelism": f"dp{world} (replicas, no collective)",
+           "cache_format": "E2M1+E4M3/16 main, MXFP4 indexer keys"}
+    if wl.pool_blocks > 0:
+        cfg["pool_blocks"] = wl.pool_blocks
+    return cfg
 
 
 def kernel_bytes(wl, n_entries):
@@ -156,15 +159,36 @@ def kernel_bytes(wl, n_entries):
       attention   per (layer, sequence) the K selected entries (256 code + 32
                   scale bytes) and their indices, the 128-token bf16 window, the
                   bf16 query, the fp32 output;
-      step        all kernels, plus the cache write of the new tokens."""
+      step        all kernels, plus the cache write of the new tokens.
+    With pools (hierarchical indexer) index_scan covers the Full layers only,
+    and topk the rest of the indexer phase: the Full layers' Top-K, the block
+    maxima (scores read, one fp32 per 8 entries written), the pool Top-K (block
+    maxima read, pool written), the Reindex layers' pool scans (per source the
+    keys of its pools' positions once, their queries, one fp32 score per
+    position written) and their Top-K (those scores read, K indices written)."""
+    from fp4_sparse_attention_pack_b200 import workloads as W
     t = wl.table
     B, H, Hi, K = wl.B, wl.H, wl.H_idx, wl.K
     scans = t.scan_layers()
     n_src = {s: sum(n_entries[s]) for s in range(t.n_sources)}
-    scanned = sorted({t.src[l] for l in scans})
-    score_bytes = sum(n_src[t.src[l]] * 4 for l in scans)
-    scan = (sum(n_src[s] * 68 for s in scanned) + len(scans) * B * Hi * (64 + 4 + 4) + score_bytes)
-    topk = score_bytes + len(scans) * B * K * 4
+    qbytes = B * Hi * (64 + 4 + 4)
+    if wl.pool_blocks > 0:
+        full = [l for l in scans if t.mode[l] == W.FULL]
+        reidx = [l for l in scans if t.mode[l] == W.REINDEX]
+        score_bytes = sum(n_src[t.src[l]] * 4 for l in full)
+        scan = sum(n_src[t.src[l]] * 68 for l in full) + len(full) * qbytes + score_bytes
+        pos = {s: sum(min(8 * wl.pool_blocks, n) for n in n_entries[s]) for s in range(t.n_sources)}
+        blocks = sum((n_src[t.src[l]] + 7) // 8 * 4 for l in full)
+        pool = score_bytes + blocks + blocks + len(full) * B * wl.pool_blocks * 4
+        pscan = (sum(pos[s] * 68 for s in sorted({t.src[l] for l in reidx})) + len(reidx) * qbytes +
+                 sum(pos[t.src[l]] * 4 for l in reidx))
+        ptopk = sum(pos[t.src[l]] * 4 for l in reidx) + len(reidx) * B * K * 4
+        topk = score_bytes + len(full) * B * K * 4 + pool + pscan + ptopk
+    else:
+        scanned = sorted({t.src[l] for l in scans})
+        score_bytes = sum(n_src[t.src[l]] * 4 for l in scans)
+        scan = (sum(n_src[s] * 68 for s in scanned) + len(scans) * qbytes + score_bytes)
+        topk = score_bytes + len(scans) * B * K * 4
     attn = 0
     for m in t.mode:
         attn += B * (WIN * 512 * 2 + H * 512 * 2 + H * 512 * 4)
@@ -380,6 +404,9 @@ def run_ours(args, rank, world, local_rank):
         for k in range(7):
             phase[k].append(e[k].elapsed_time(e[k + 1]))
     phase_ms = {n: statistics.mean(v) for n, v in zip(names, phase)}
+    if wl.pool_blocks > 0:
+        phase_note = ("hierarchical indexer: index_scan = the Full layers' scans; topk = their Top-K, "
+                      "the pool build and the Reindex layers' pool scans with their Top-K")
 
     # End to end: every step copies its inputs from pinned host memory and reads its
     # outputs back, through csa2_layer_step.  Two device buffer sets and two copy
@@ -462,6 +489,7 @@ def run_ours(args, rank, world, local_rank):
                      "launch_ms": phase_ms[dom]},
         "kernels": kernels,
         "phase_ms": phase_ms,
+        **({"phase_note": phase_note} if wl.pool_blocks > 0 else {}),
         "e2e": {"value": L * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "method": "csa2_layer_step with every step's inputs copied from pinned host memory and "

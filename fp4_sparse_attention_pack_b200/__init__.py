@@ -13,13 +13,15 @@ import os
 from ._build import LIB
 
 __all__ = ["Csa2Error", "lib", "csa2_cache", "csa2_window", "csa2_model", "csa2_step_in",
-           "csa2_step_out", "pack_cache", "index_topk", "index_topk_workspace", "sparse_attn",
+           "csa2_step_out", "pack_cache", "index_topk", "index_topk_workspace", "index_pool_workspace",
+           "index_topk_pool", "index_topk_in_pool", "POOL_BLOCK", "MAX_POOL_BLOCKS", "sparse_attn",
            "sparse_attn_workspace", "window_append", "layer_step", "layer_step_workspace", "layer_step_launches", "seq_image_bytes", "cache_export",
            "cache_import",
            "SWA_ONLY", "FULL", "REINDEX", "REUSE", "DTYPE_BF16", "DTYPE_F32"]
 
 SWA_ONLY, FULL, REINDEX, REUSE = 0, 1, 2, 3
 DTYPE_BF16, DTYPE_F32 = 0, 1
+POOL_BLOCK, MAX_POOL_BLOCKS = 8, 8192
 DEVERR_CAPACITY, DEVERR_PAGE, DEVERR_COUNT, DEVERR_TIMEOUT, DEVERR_IMAGE = 1, 2, 4, 8, 16
 
 _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
@@ -47,7 +49,7 @@ class csa2_model(ctypes.Structure):
                 ("src", ctypes.POINTER(_i32)), ("idx_src", ctypes.POINTER(_i32)),
                 ("caches", ctypes.POINTER(csa2_cache)), ("w_idx", ctypes.POINTER(_vp)),
                 ("windows", ctypes.POINTER(csa2_window)), ("batch", _i32), ("H", _i32),
-                ("H_idx", _i32), ("K", _i32), ("scale", _f32)]
+                ("H_idx", _i32), ("K", _i32), ("scale", _f32), ("pool_blocks", _i32)]
 
 
 class csa2_step_in(ctypes.Structure):
@@ -78,6 +80,11 @@ def lib():
             ("csa2_index_topk_workspace", _sz, [ctypes.c_int] * 4),
             ("csa2_index_topk", ctypes.c_int, [P(csa2_cache), _vp, _vp, ctypes.c_int, ctypes.c_int, _vp,
                                                _vp, _vp, _sz, _vp]),
+            ("csa2_index_pool_workspace", _sz, [ctypes.c_int] * 5),
+            ("csa2_index_topk_pool", ctypes.c_int, [P(csa2_cache), _vp, _vp, ctypes.c_int, ctypes.c_int, _vp,
+                                                    _vp, ctypes.c_int, _vp, _vp, _sz, _vp]),
+            ("csa2_index_topk_in_pool", ctypes.c_int, [P(csa2_cache), _vp, _vp, ctypes.c_int, ctypes.c_int,
+                                                       _vp, ctypes.c_int, _vp, _vp, _vp, _sz, _vp]),
             ("csa2_sparse_attn_workspace", _sz, [ctypes.c_int] * 3),
             ("csa2_sparse_attn", ctypes.c_int, [P(csa2_cache), _vp, ctypes.c_int, _vp, ctypes.c_int,
                                                 P(csa2_window), ctypes.c_float, _vp, _vp, _sz, _vp]),
@@ -130,6 +137,29 @@ def index_topk(cache: csa2_cache, q_idx, w, K: int, idx_out, ws, score_out=None,
     _ok(lib().csa2_index_topk(ctypes.byref(cache), _ptr(q_idx), _ptr(w), H_idx, K, _ptr(idx_out),
                               _ptr(score_out), _ptr(ws), ws.numel() * ws.element_size(),
                               _stream(stream)), "csa2_index_topk")
+
+
+def index_pool_workspace(batch: int, max_entries: int, H_idx: int, K: int, pool_blocks: int) -> int:
+    return int(lib().csa2_index_pool_workspace(batch, max_entries, H_idx, K, pool_blocks))
+
+
+def index_topk_pool(cache: csa2_cache, q_idx, w, K: int, idx_out, pool_out, ws, score_out=None,
+                    stream=None):
+    """Full-layer scan: Top-K into idx_out and the block pool into pool_out
+    [batch][pool_blocks]."""
+    H_idx = q_idx.shape[1]
+    _ok(lib().csa2_index_topk_pool(ctypes.byref(cache), _ptr(q_idx), _ptr(w), H_idx, K, _ptr(idx_out),
+                                   _ptr(score_out), pool_out.shape[1], _ptr(pool_out), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)), "csa2_index_topk_pool")
+
+
+def index_topk_in_pool(cache: csa2_cache, q_idx, w, K: int, pool, idx_out, ws, score_out=None, stream=None):
+    """Scan restricted to pool [batch][pool_blocks]; Top-K into idx_out."""
+    H_idx = q_idx.shape[1]
+    _ok(lib().csa2_index_topk_in_pool(ctypes.byref(cache), _ptr(q_idx), _ptr(w), H_idx, K, _ptr(pool),
+                                      pool.shape[1], _ptr(idx_out), _ptr(score_out), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)),
+        "csa2_index_topk_in_pool")
 
 
 def sparse_attn_workspace(batch: int, H: int, K: int) -> int:

@@ -118,6 +118,118 @@ int csa2_index_topk(const csa2_cache* cache, const uint16_t* q_idx, const float*
     return cuda_status(launch_index_topk(sb, (cudaStream_t)stream));
 }
 
+// ---------------------------------------------------------------- hierarchical indexer
+
+namespace {
+
+// Workspace of the standalone pool calls: one scan problem whose score rows hold
+// max(max_entries, 8 * pool_blocks) floats, the block-maximum rows, pool_n.
+struct PoolWs {
+    size_t scan, bmax, count, total;
+    int rows;
+    int64_t bstride;
+};
+
+PoolWs pool_ws(int batch, int max_entries, int H_idx, int pool_blocks) {
+    PoolWs w;
+    w.rows = std::max(max_entries, kPoolBlock * pool_blocks);
+    w.bstride = block_row_stride(max_entries);
+    w.scan = align_up(topk_ws_one(batch, w.rows, H_idx));
+    w.bmax = align_up((size_t)batch * w.bstride * sizeof(float));
+    w.count = align_up((size_t)batch * sizeof(int32_t));
+    w.total = w.scan + w.bmax + w.count;
+    return w;
+}
+
+int check_scan_args(const csa2_cache* cache, const uint16_t* q_idx, const float* w, int H_idx, int K,
+                    const int32_t* idx_out, const float* score_out, int pool_blocks, const int32_t* pool,
+                    const void* ws) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (H_idx < 1 || H_idx > CSA2_MAX_H_IDX || K < 1 || K > CSA2_MAX_K) return CSA2_ERR_INVALID_ARG;
+    if (pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS) return CSA2_ERR_INVALID_ARG;
+    if (!q_idx || !w || !idx_out || !pool) return CSA2_ERR_INVALID_ARG;
+    if (!a16(q_idx) || !a16(w) || !a16(idx_out) || (score_out && !a16(score_out)) || !a16(pool) ||
+        (ws && !a16(ws)))
+        return CSA2_ERR_ALIGN;
+    return CSA2_OK;
+}
+
+}  // namespace
+
+size_t csa2_index_pool_workspace(int batch, int max_entries, int H_idx, int K, int pool_blocks) {
+    (void)K;
+    if (batch < 1 || max_entries < 0 || H_idx < 1 || pool_blocks < 1 || pool_blocks > CSA2_MAX_POOL_BLOCKS)
+        return 0;
+    return pool_ws(batch, max_entries, H_idx, pool_blocks).total;
+}
+
+int csa2_index_topk_pool(const csa2_cache* cache, const uint16_t* q_idx, const float* w, int H_idx, int K,
+                         int32_t* idx_out, float* score_out, int pool_blocks, int32_t* pool_out, void* ws,
+                         size_t ws_bytes, csa2_stream stream) {
+    int rc = check_scan_args(cache, q_idx, w, H_idx, K, idx_out, score_out, pool_blocks, pool_out, ws);
+    if (rc) return rc;
+    const int cap = cache->max_pages * PAGE;
+    const PoolWs pw = pool_ws(cache->batch, cap, H_idx, pool_blocks);
+    if (!ws || ws_bytes < pw.total) return CSA2_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* wsp = static_cast<uint8_t*>(ws);
+    ScanBatch sb;
+    std::memset(&sb, 0, sizeof(sb));
+    sb.n = 1;
+    sb.H_idx = H_idx;
+    sb.K = K;
+    sb.p[0].cache = view_of(*cache);
+    sb.p[0].q_idx = q_idx;
+    sb.p[0].w = w;
+    sb.p[0].idx_out = idx_out;
+    sb.p[0].score_out = score_out;
+    carve_scan_workspace(sb, wsp, cache->batch, pw.rows);
+    rc = cuda_status(launch_index_topk(sb, st));
+    if (rc) return rc;
+    float* bmax = reinterpret_cast<float*>(wsp + pw.scan);
+    rc = cuda_status(launch_block_max(sb, bmax, pw.bstride, st));
+    if (rc) return rc;
+    ScanBatch sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.n = 1;
+    sp.H_idx = H_idx;
+    sp.K = pool_blocks;
+    sp.score_stride = pw.bstride;
+    sp.p[0].cache = sb.p[0].cache;
+    sp.p[0].scores = bmax;
+    sp.p[0].block_rows = 1;
+    sp.p[0].idx_out = pool_out;
+    return cuda_status(launch_topk(sp, st));
+}
+
+int csa2_index_topk_in_pool(const csa2_cache* cache, const uint16_t* q_idx, const float* w, int H_idx, int K,
+                            const int32_t* pool, int pool_blocks, int32_t* idx_out, float* score_out, void* ws,
+                            size_t ws_bytes, csa2_stream stream) {
+    int rc = check_scan_args(cache, q_idx, w, H_idx, K, idx_out, score_out, pool_blocks, pool, ws);
+    if (rc) return rc;
+    const int cap = cache->max_pages * PAGE;
+    const PoolWs pw = pool_ws(cache->batch, cap, H_idx, pool_blocks);
+    if (!ws || ws_bytes < pw.total) return CSA2_ERR_WORKSPACE;
+    uint8_t* wsp = static_cast<uint8_t*>(ws);
+    ScanBatch sb;
+    std::memset(&sb, 0, sizeof(sb));
+    sb.n = 1;
+    sb.H_idx = H_idx;
+    sb.K = K;
+    ScanProblem& P = sb.p[0];
+    P.cache = view_of(*cache);
+    P.q_idx = q_idx;
+    P.w = w;
+    P.idx_out = idx_out;
+    P.score_out = score_out;
+    P.pool = pool;
+    P.pool_blocks = pool_blocks;
+    P.pool_n = reinterpret_cast<int32_t*>(wsp + pw.scan + pw.bmax);
+    carve_scan_workspace(sb, wsp, cache->batch, pw.rows);
+    return cuda_status(launch_index_topk(sb, (cudaStream_t)stream));
+}
+
 size_t csa2_sparse_attn_workspace(int batch, int H, int K) {
     if (batch < 1 || H < 1 || K < 0) return 0;
     return attn_workspace_bytes(1, batch, H, K);
@@ -189,7 +301,7 @@ int check_model(const csa2_model* m) {
         !m->w_idx || !m->windows)
         return CSA2_ERR_INVALID_ARG;
     if (m->batch < 1 || m->H < 1 || m->H > CSA2_MAX_H || m->H_idx < 1 || m->H_idx > CSA2_MAX_H_IDX ||
-        m->K < 1 || m->K > CSA2_MAX_K)
+        m->K < 1 || m->K > CSA2_MAX_K || m->pool_blocks < 0 || m->pool_blocks > CSA2_MAX_POOL_BLOCKS)
         return CSA2_ERR_INVALID_ARG;
     int full_of[CSA2_MAX_SOURCES];
     for (int s = 0; s < m->n_sources; ++s) full_of[s] = -1;
@@ -237,12 +349,46 @@ int n_scans(const csa2_model* m) {
     return n;
 }
 
+int n_mode(const csa2_model* m, int mode) {
+    int n = 0;
+    for (int l = 0; l < m->n_layers; ++l) n += m->mode[l] == mode;
+    return n;
+}
+
+// Step workspace, in order: scan workspace (one region; with pools one for the
+// FULL layers and one for the REINDEX layers), attention partials, and with
+// pools the pools [n_sources][batch][pool_blocks], the block-maximum rows of the
+// FULL layers and pool_n of the REINDEX layers.
+struct StepWs {
+    size_t scan1, scan2, attn, pools, bmax, count, total;
+    int rows;
+    int64_t bstride;
+};
+
+StepWs step_ws(const csa2_model* m) {
+    StepWs w{};
+    const int cap = max_entries(m), B = m->batch, PB = m->pool_blocks;
+    w.rows = PB > 0 ? std::max(cap, kPoolBlock * PB) : cap;
+    w.bstride = block_row_stride(cap);
+    if (PB == 0) {
+        w.scan1 = align_up(scan_workspace_bytes(n_scans(m), B, cap, m->H_idx));
+    } else {
+        w.scan1 = align_up(scan_workspace_bytes(n_mode(m, CSA2_MODE_FULL), B, w.rows, m->H_idx));
+        w.scan2 = align_up(scan_workspace_bytes(n_mode(m, CSA2_MODE_REINDEX), B, w.rows, m->H_idx));
+        w.pools = align_up((size_t)m->n_sources * B * PB * sizeof(int32_t));
+        w.bmax = align_up((size_t)n_mode(m, CSA2_MODE_FULL) * B * w.bstride * sizeof(float));
+        w.count = align_up((size_t)n_mode(m, CSA2_MODE_REINDEX) * B * sizeof(int32_t));
+    }
+    w.attn = align_up(attn_workspace_bytes(m->n_layers, B, m->H, m->K));
+    w.total = w.scan1 + w.scan2 + w.attn + w.pools + w.bmax + w.count;
+    return w;
+}
+
 }  // namespace
 
 size_t csa2_layer_step_workspace(const csa2_model* m) {
     if (check_model(m)) return 0;
-    return align_up(scan_workspace_bytes(n_scans(m), m->batch, max_entries(m), m->H_idx)) +
-           align_up(attn_workspace_bytes(m->n_layers, m->batch, m->H, m->K));
+    return step_ws(m).total;
 }
 
 namespace {
@@ -324,16 +470,18 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
     }
     if (ev) cudaEventRecord(ev[2], st);
 
-    // (3) every Full / Reindex layer scans its source with its own query
+    // (3) every Full / Reindex layer scans its source with its own query; with
+    // pools the Full layers go first and build their sources' pools
     uint8_t* wsp = static_cast<uint8_t*>(ws);
-    const int cap = max_entries(m);
+    const StepWs sw = step_ws(m);
+    const int PB = m->pool_blocks;
     ScanBatch sb;
     std::memset(&sb, 0, sizeof(sb));
     sb.H_idx = m->H_idx;
     sb.K = m->K;
     for (int l = 0; l < L; ++l) {
         const int md = m->mode[l];
-        if (md != CSA2_MODE_FULL && md != CSA2_MODE_REINDEX) continue;
+        if (md != CSA2_MODE_FULL && (md != CSA2_MODE_REINDEX || PB > 0)) continue;
         ScanProblem& P = sb.p[sb.n++];
         P.cache = view_of(m->caches[m->src[l]]);
         P.q_idx = in->q_idx[l];
@@ -341,19 +489,69 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
         P.idx_out = out->idx[l];
         P.score_out = nullptr;
     }
-    carve_scan_workspace(sb, wsp, B, cap);
-    wsp += align_up(scan_workspace_bytes(sb.n, B, cap, m->H_idx));
+    carve_scan_workspace(sb, wsp, B, sw.rows);
     if (sb.n > 0) {
         rc = cuda_status(launch_index_topk(sb, st, ev ? ev + 3 : nullptr));
         if (rc) return rc;
     } else if (ev) {
         for (int i = 3; i < 6; ++i) cudaEventRecord(ev[i], st);
     }
+    if (PB > 0) {
+        uint8_t* region = wsp + sw.scan1 + sw.scan2 + sw.attn;
+        int32_t* pools = reinterpret_cast<int32_t*>(region);
+        float* bmax = reinterpret_cast<float*>(region + sw.pools);
+        int32_t* pool_n = reinterpret_cast<int32_t*>(region + sw.pools + sw.bmax);
+        // the pool of each source: block maxima of its Full layer's scores, their Top-K
+        rc = cuda_status(launch_block_max(sb, bmax, sw.bstride, st));
+        if (rc) return rc;
+        ScanBatch sp;
+        std::memset(&sp, 0, sizeof(sp));
+        sp.n = sb.n;
+        sp.H_idx = m->H_idx;
+        sp.K = PB;
+        sp.score_stride = sw.bstride;
+        int li = 0;
+        for (int l = 0; l < L; ++l) {
+            if (m->mode[l] != CSA2_MODE_FULL) continue;
+            ScanProblem& P = sp.p[li];
+            P.cache = sb.p[li].cache;
+            P.scores = bmax + (int64_t)li * B * sw.bstride;
+            P.block_rows = 1;
+            P.idx_out = pools + (int64_t)m->src[l] * B * PB;
+            ++li;
+        }
+        rc = cuda_status(launch_topk(sp, st));
+        if (rc) return rc;
+        // the Reindex layers over their sources' pools
+        ScanBatch sr;
+        std::memset(&sr, 0, sizeof(sr));
+        sr.H_idx = m->H_idx;
+        sr.K = m->K;
+        for (int l = 0; l < L; ++l) {
+            if (m->mode[l] != CSA2_MODE_REINDEX) continue;
+            ScanProblem& P = sr.p[sr.n];
+            P.cache = view_of(m->caches[m->src[l]]);
+            P.q_idx = in->q_idx[l];
+            P.w = in->w[l];
+            P.idx_out = out->idx[l];
+            P.pool = pools + (int64_t)m->src[l] * B * PB;
+            P.pool_blocks = PB;
+            P.pool_n = pool_n + (int64_t)sr.n * B;
+            ++sr.n;
+        }
+        if (sr.n > 0) {
+            carve_scan_workspace(sr, wsp + sw.scan1, B, sw.rows);
+            rc = cuda_status(launch_index_topk(sr, st));
+            if (rc) return rc;
+        }
+        if (ev) cudaEventRecord(ev[5], st);  // the indexer phase ends after the pool scans
+    }
+    wsp += sw.scan1 + sw.scan2;
 
     // (4) every layer attends; Reuse layers read the indices of idx_src
     AttnBatch ab;
     model_attn_batch(m, ab);
-    const size_t units = attn_workspace_bytes(L, B, m->H, m->K) / ((D + 2) * sizeof(float));
+    const size_t units = attn_workspace_bytes(L, B, m->H, m->K) / ((D + 2) * sizeof(float));  // in wsp
     ab.part_o = reinterpret_cast<float*>(wsp);
     ab.part_ml = ab.part_o + units * D;
     for (int l = 0; l < L; ++l) {
@@ -396,6 +594,10 @@ int csa2_layer_step_launches(const csa2_model* m, const csa2_step_in* in) {
             break;
         }
     if (n_scans(m) > 0) n += 3;  // query quantisation, scan, Top-K
+    if (m->pool_blocks > 0) {
+        n += 2;                                        // block maxima, pool Top-K
+        if (n_mode(m, CSA2_MODE_REINDEX) > 0) n += 4;  // pool count, quantisation, scan, Top-K
+    }
     AttnBatch ab;
     model_attn_batch(m, ab);
     return n + sparse_attn_launches(ab);

@@ -25,6 +25,15 @@ struct ScanProblem {
     float* scores;          // workspace: fp32 [batch][score_stride]
     int32_t* idx_out;       // [batch][K]
     float* score_out;       // nullable [batch][K]
+    // Hierarchical indexer.  pool (nullable): [batch][pool_blocks] ids of
+    // 8-entry blocks, increasing, -1 padded.  The problem then scores only the
+    // pool's entries: position i of its score row is entry 8 * pool[i / 8] + i % 8,
+    // and pool_n[b] (written by launch_pool_count) is the number of valid
+    // positions, a prefix of the row.
+    const int32_t* pool;
+    int32_t* pool_n;        // [batch]
+    int pool_blocks;
+    int block_rows;         // the score row holds block maxima: ceil(n_entries / 8) of them
 };
 
 constexpr int kMaxProblems = 64;
@@ -38,6 +47,20 @@ struct ScanBatch {
     int K;
 };
 
+constexpr int kPoolBlock = 8;  // entries per hierarchical-indexer block
+
+// Length of problem P's score row for sequence b.
+__device__ __forceinline__ int row_len(const ScanProblem& P, int b) {
+    if (P.pool) return P.pool_n[b];
+    const int n = entries_of(P.cache, b);
+    return P.block_rows ? (n + kPoolBlock - 1) / kPoolBlock : n;
+}
+
+// Entry (or block id) at position i of problem P's score row for sequence b.
+__device__ __forceinline__ int row_entry(const ScanProblem& P, int b, int i) {
+    return P.pool ? kPoolBlock * P.pool[(int64_t)b * P.pool_blocks + i / kPoolBlock] + i % kPoolBlock : i;
+}
+
 // Bytes of scan workspace for n problems.
 size_t scan_workspace_bytes(int n_problems, int batch, int max_entries, int H_idx);
 // Point sb.qc / sb.qs / every problem's scores into ws (sb.n must be set).
@@ -46,6 +69,22 @@ void carve_scan_workspace(ScanBatch& sb, uint8_t* ws, int batch, int max_entries
 // ev (nullable): events recorded after query quantisation, after the scan and
 // after Top-K (three cudaEvent_t).
 cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t* ev = nullptr);
+// Kernel launches one launch_index_topk(sb) call makes.
+int index_topk_launches(const ScanBatch& sb);
+
+// Top-K of every problem's score row (row_len positions), sb.K per row.
+cudaError_t launch_topk(const ScanBatch& sb, cudaStream_t st);
+
+// pool_n of every pool problem of sb: the valid prefix of its positions.
+cudaError_t launch_pool_count(const ScanBatch& sb, cudaStream_t st);
+
+// Block maxima of every problem's score row: bmax[(i * batch + b) * bstride + j]
+// = max of entries 8j .. 8j + 7 (below n_entries) of problem i, sequence b.
+// bstride is a multiple of 4.
+cudaError_t launch_block_max(const ScanBatch& sb, float* bmax, int64_t bstride, cudaStream_t st);
+inline int64_t block_row_stride(int max_entries) {
+    return ((int64_t)(max_entries + kPoolBlock - 1) / kPoolBlock + 3) / 4 * 4;
+}
 
 // ---- attention
 struct AttnProblem {

@@ -10,7 +10,8 @@
 // CUDA-core scan: one thread per entry.  E2M1 values times 2 are the integers
 // {0,1,2,3,4,6,8,12} (with sign), so each 32-channel block product is an exact
 // int32 dot of int8 vectors (dp4a); the block's two E8M0 scales are applied to
-// that exact integer and the four blocks summed in fp32.  Keys stream with
+// that exact integer and the four blocks summed in fp32.  A problem with a
+// pool (hierarchical indexer) runs one thread per pool position instead.  Keys stream with
 // 16-byte loads and an evict-first L2 policy (each key is read once per scan).
 #include "common.cuh"
 #include "kernels.cuh"
@@ -111,9 +112,10 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_cuda(ScanBatch sb) {
     for (int i = threadIdx.x; i < H; i += blockDim.x) wv[i] = P.w[(int64_t)b * H + i];
     __syncthreads();
 
-    const int n = entries_of(P.cache, b);
-    const int e = blockIdx.x * kScanThreads + threadIdx.x;
-    if (e >= n) return;
+    // position i of the score row; entry e = i unless the problem scans a pool
+    const int i = blockIdx.x * kScanThreads + threadIdx.x;
+    if (i >= row_len(P, b)) return;
+    const int e = row_entry(P, b, i);
     const int p = page_of(P.cache, b, e);
     if (p < 0) return;
     const int64_t ent = (int64_t)p * PAGE + (e % PAGE);
@@ -151,12 +153,11 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_cuda(ScanBatch sb) {
         }
         score = fmaf(wv[h], fmaxf(dot, 0.0f), score);
     }
-    P.scores[(int64_t)b * sb.score_stride + e] = score;
+    P.scores[(int64_t)b * sb.score_stride + i] = score;
 }
 
 }  // namespace
 
-cudaError_t launch_topk(const ScanBatch& sb, cudaStream_t st);
 bool scan_mma_supported(const ScanBatch& sb);
 cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st);
 
@@ -180,8 +181,22 @@ void carve_scan_workspace(ScanBatch& sb, uint8_t* ws, int batch, int max_entries
         sb.p[i].scores = reinterpret_cast<float*>(ws) + (size_t)i * batch * max_entries;
 }
 
+namespace {
+bool has_pool(const ScanBatch& sb) {
+    for (int i = 0; i < sb.n; ++i)
+        if (sb.p[i].pool) return true;
+    return false;
+}
+}  // namespace
+
+int index_topk_launches(const ScanBatch& sb) { return 3 + (has_pool(sb) ? 1 : 0); }
+
 cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t* ev) {
     const int batch = sb.p[0].cache.batch;
+    if (has_pool(sb)) {
+        cudaError_t e = launch_pool_count(sb, st);
+        if (e != cudaSuccess) return e;
+    }
     {
         const int total = batch * sb.H_idx * 4;
         dim3 grid((total + 127) / 128, sb.n);
@@ -195,8 +210,9 @@ cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t*
         if (e != cudaSuccess) return e;
         if (ev) cudaEventRecord(ev[1], st);
     } else {
-        int cap = 0;
-        for (int i = 0; i < sb.n; ++i) cap = max(cap, sb.p[i].cache.max_pages * PAGE);
+        int cap = 0;  // positions per score row at most
+        for (int i = 0; i < sb.n; ++i)
+            cap = max(cap, sb.p[i].pool ? kPoolBlock * sb.p[i].pool_blocks : sb.p[i].cache.max_pages * PAGE);
         dim3 grid((cap + kScanThreads - 1) / kScanThreads, batch, sb.n);
         const size_t smem = (size_t)sb.H_idx * (32 + 4 + 1) * 4;
         k_scan_cuda<<<grid, kScanThreads, smem, st>>>(sb);

@@ -30,6 +30,9 @@
 //           landed in accumulator g.  Warp w of a group reads TMEM lane quadrant
 //           w % 4 and problem (w / 4) % 2 of the pass: tcgen05.ld of the 64 head
 //           columns of its entry, ReLU, weight, sum, one score store.
+//           A subset that scans a pool (hierarchical indexer) instead gathers
+//           each tile as 16 boxes of 8 rows, one per pool block, each into its
+//           own 512-byte slot, so the swizzled layout is that of a whole page.
 //   warp 18 scale warp: rearranges the E8M0 scales that landed in shared memory
 //           into the 32x128-bit layout tcgen05.cp reads (per item for the
 //           queries, per stage for the keys) and signals them ready, keeping
@@ -77,11 +80,13 @@ struct ScanSub {
     int chunk;    // tiles per work item
     int chunks;   // work items per sequence
     int item0;    // first work item
+    int pool;     // the problems scan the same pool (positions instead of entries)
     int8_t prob[kMaxSub];
 };
 
 struct MmaScanMaps {
     CUtensorMap keys[kMaxSources];  // per distinct cache: idx codes [num_pages*64][64 B]
+    CUtensorMap keys8[kMaxSources]; // the same with 8-row boxes (pool blocks)
     CUtensorMap queries;            // [n * batch * 64][64 B]
     ScanSub sub[kMaxProblems];
     int n_sub;
@@ -97,6 +102,7 @@ struct __align__(1024) Smem {
     uint8_t sfb_tc[2][kMaxPasses][512];
     float w[2][kMaxSub][kHeads];
     float* rows[2][kMaxSub];                 // score row of the item's sequence, per problem
+    int prow[kMaxChunk * 16];                // pool items: first physical key row of each slot
     uint64_t full[kStages], empty[kStages], sfa_ready[kStages];
     uint64_t bfull[2], bempty[2], sfb_ready[2];
     uint64_t tfull[kGroups], tempty[kGroups];
@@ -119,7 +125,8 @@ __device__ __forceinline__ bool item_at(const ScanBatch& sb, const MmaScanMaps& 
     it.s = s;
     it.b = r / S.chunks;
     const int c = r - it.b * S.chunks;
-    it.n = entries_of(sb.p[S.prob[0]].cache, it.b);
+    const ScanProblem& P0 = sb.p[S.prob[0]];
+    it.n = S.pool ? min(max(P0.pool_n[it.b], 0), kPoolBlock * P0.pool_blocks) : entries_of(P0.cache, it.b);
     const int tiles = (it.n + kTile - 1) / kTile;
     it.t0 = c * S.chunk;
     it.t1 = min(it.t0 + S.chunk, tiles);
@@ -204,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int used_pages = (it.n + PAGE - 1) / PAGE;
             const int li = 2 * it.t0 + lane;  // logical page this lane looks up
             int my_pg = -1;
-            if (lane < 2 * (it.t1 - it.t0) && li < used_pages) {
+            if (!S.pool && lane < 2 * (it.t1 - it.t0) && li < used_pages) {
                 const int pp = c.page_table[(int64_t)it.b * c.max_pages + li];
                 if (pp >= 0 && pp < c.num_pages)
                     my_pg = pp;
@@ -231,13 +238,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (++bslot == 2) bslot = 0, bphase ^= 1;
             const CUtensorMap* kmap = &mp.keys[S.src];
+            if (S.pool) {
+                // physical first row of every pool block of the item (positions
+                // below it.n are valid, so their blocks lie below n_entries)
+                const ScanProblem& P0 = sb.p[S.prob[0]];
+                const int slots = (it.n + kPoolBlock - 1) / kPoolBlock;
+                __syncwarp();  // the previous item's reads of prow are done
+                for (int i = lane; i < 16 * (it.t1 - it.t0); i += 32) {
+                    const int slot = 16 * it.t0 + i;
+                    int r = -1;
+                    if (slot < slots) {
+                        const int e0 = kPoolBlock * P0.pool[(int64_t)it.b * P0.pool_blocks + slot];
+                        const int pp = c.page_table[(int64_t)it.b * c.max_pages + e0 / PAGE];
+                        if (pp >= 0 && pp < c.num_pages)
+                            r = pp * PAGE + e0 % PAGE;
+                        else
+                            atomicOr(c.status, CSA2_DEVERR_PAGE);
+                    }
+                    sm.prow[i] = r;
+                }
+                __syncwarp();
+            }
             for (int t = it.t0; t < it.t1 && !stop; ++t) {
                 const int pg0 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0));
                 const int pg1 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0) + 1);
+                const int prow = S.pool && lane < 16 ? sm.prow[16 * (t - it.t0) + lane] : -1;
+                const unsigned have = __ballot_sync(0xffffffffu, prow >= 0);
                 if (!mbar_wait_warp(&sm.empty[stage], sphase ^ 1)) {
                     if (lane == 0) raise_abort(sm, c.status);
                     stop = true;
                     break;
+                }
+                if (S.pool) {
+                    if (have == 0) {
+                        mbar_arrive_w(&sm.full[stage]);
+                    } else {
+                        mbar_expect_tx_w(&sm.full[stage], __popc(have) * kPoolBlock * (ICB + ISB));
+                        __syncwarp();
+                        if (prow >= 0) {
+                            tma_load_2d(sm.a[stage] + lane * kPoolBlock * ICB, &mp.keys8[S.src], 0, prow,
+                                        &sm.full[stage], pol_stream);
+                            bulk_load(sm.sfa_raw[stage] + lane * kPoolBlock * ISB, c.idx_scales + (int64_t)prow * ISB,
+                                      kPoolBlock * ISB, &sm.full[stage], pol_stream);
+                        }
+                    }
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (sphase << stage);
+                    if (++stage == kStages) stage = 0, sphase ^= 1;
+                    continue;
                 }
                 const uint32_t bytes = (pg0 >= 0 ? PAGE * (ICB + ISB) : 0) + (pg1 >= 0 ? PAGE * (ICB + ISB) : 0);
                 if (bytes == 0) {
@@ -481,6 +529,7 @@ cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st) {
     const uint8_t* seen[kMaxSources];
     int src_of[kMaxProblems];
     int cap_tiles[kMaxSources];
+    bool have8[kMaxSources] = {};
     for (int i = 0; i < sb.n; ++i) {
         const CacheView& c = sb.p[i].cache;
         int j = 0;
@@ -494,20 +543,36 @@ cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st) {
             ++srcs;
         }
         src_of[i] = j;
+        if (sb.p[i].pool && !have8[j]) {
+            if (!make_rows64_map(&mp.keys8[j], c.idx_codes, (uint64_t)c.num_pages * PAGE, kPoolBlock))
+                return cudaErrorInvalidValue;
+            have8[j] = true;
+        }
     }
-    for (int j = 0; j < srcs; ++j) {
+    // groups: problems over one cache that scan the same pool (or none)
+    bool grouped[kMaxProblems] = {};
+    int sub_tiles[kMaxProblems];
+    for (int i0 = 0; i0 < sb.n; ++i0) {
+        if (grouped[i0]) continue;
         int members[kMaxProblems], m = 0;
-        for (int i = 0; i < sb.n; ++i)
-            if (src_of[i] == j) members[m++] = i;
+        for (int i = i0; i < sb.n; ++i)
+            if (!grouped[i] && src_of[i] == src_of[i0] && sb.p[i].pool == sb.p[i0].pool) {
+                members[m++] = i;
+                grouped[i] = true;
+            }
+        const bool pool = sb.p[i0].pool != nullptr;
+        const int tiles = pool ? (kPoolBlock * sb.p[i0].pool_blocks + kTile - 1) / kTile : cap_tiles[src_of[i0]];
         // split into near-equal subsets of at most kMaxSub problems
         const int parts = (m + kMaxSub - 1) / kMaxSub;
-        for (int q = 0, i0 = 0; q < parts; ++q) {
-            const int cnt = (m - i0) / (parts - q);
+        for (int q = 0, k0 = 0; q < parts; ++q) {
+            const int cnt = (m - k0) / (parts - q);
+            sub_tiles[mp.n_sub] = tiles;
             ScanSub& S = mp.sub[mp.n_sub++];
-            S.src = j;
+            S.src = src_of[i0];
+            S.pool = pool ? 1 : 0;
             S.n = cnt;
-            for (int k = 0; k < cnt; ++k) S.prob[k] = (int8_t)members[i0 + k];
-            i0 += cnt;
+            for (int k = 0; k < cnt; ++k) S.prob[k] = (int8_t)members[k0 + k];
+            k0 += cnt;
         }
     }
     // Tiles per work item: about 64 tile-problems of work each (so subsets of
@@ -520,7 +585,7 @@ cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st) {
         for (int s = 0; s < mp.n_sub; ++s) {
             ScanSub& S = mp.sub[s];
             S.chunk = std::max(2, std::min(kMaxChunk, base / S.n));
-            S.chunks = (cap_tiles[S.src] + S.chunk - 1) / S.chunk;
+            S.chunks = (sub_tiles[s] + S.chunk - 1) / S.chunk;
             S.item0 = items;
             items += batch * S.chunks;
         }

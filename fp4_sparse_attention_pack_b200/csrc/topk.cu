@@ -1,7 +1,10 @@
 // Per-sequence Top-K of the indexer scores ("n'en garde que les 512 meilleures").
 //
 // Scores map to order-preserving uint32 keys; the K largest are kept, equal
-// scores lower index first, and written in increasing index order.
+// scores lower index first, and written in increasing index order.  A row is a
+// problem's score row (entries), its pool positions (hierarchical indexer: the
+// winners are written as the entries they stand for), or its block maxima
+// (pool build: the winners are block ids).
 //
 // One CTA of 512 threads per (problem, sequence):
 //   1. Threshold guess: 2,048 strided samples of the row; an exact radix select
@@ -116,10 +119,10 @@ __device__ void radix_select(KeyAt key_at, int cnt, int k, TopkSmem& sm, uint32_
 }
 
 // Ordered compaction of the Top-K: keys above kth, then (in index order) the
-// first `need` keys equal to it.  Writes out positions [0, K).  Each thread
-// takes a contiguous run of kRun keys per round.
-template <class KeyAt, class IdxAt>
-__device__ void emit_topk(KeyAt key_at, IdxAt idx_at, int cnt, uint32_t kth, int need, int K,
+// first `need` keys equal to it.  Writes out positions [0, K), each as
+// out_of(row position).  Each thread takes a contiguous run of kRun keys per round.
+template <class KeyAt, class IdxAt, class OutOf>
+__device__ void emit_topk(KeyAt key_at, IdxAt idx_at, OutOf out_of, int cnt, uint32_t kth, int need, int K,
                           TopkSmem& sm, int32_t* io, float* so) {
     int base_out = 0, eq_seen = 0;
     for (int base = 0; base < cnt; base += kThreads * kRun) {
@@ -149,7 +152,7 @@ __device__ void emit_topk(KeyAt key_at, IdxAt idx_at, int cnt, uint32_t kth, int
             }
             if (take) {
                 if (o < K) {
-                    io[o] = idx_at(i0 + v);
+                    io[o] = out_of(idx_at(i0 + v));
                     if (so) so[o] = order_key_f32(kk[v]);
                 }
                 ++o;
@@ -167,15 +170,16 @@ __global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanB
     const ScanProblem& P = sb.p[blockIdx.y];
     const int b = blockIdx.x;
     const int K = sb.K;
-    const int n = entries_of(P.cache, b);
+    const int n = row_len(P, b);
     const float* row = P.scores + (int64_t)b * sb.score_stride;
     int32_t* io = P.idx_out + (int64_t)b * K;
     float* so = P.score_out ? P.score_out + (int64_t)b * K : nullptr;
     const int tid = threadIdx.x;
+    auto out_of = [&](int i) { return row_entry(P, b, i); };
 
     if (n <= K) {
         for (int i = tid; i < K; i += kThreads) {
-            io[i] = i < n ? i : -1;
+            io[i] = i < n ? out_of(i) : -1;
             if (so) so[i] = i < n ? row[i] : 0.0f;
         }
         return;
@@ -241,13 +245,13 @@ __global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanB
     if (fits && cnt >= K) {
         // 3. exact selection among the candidates (already in index order)
         radix_select([&](int i) { return sm.key[i]; }, cnt, K, sm, &kth, &need);
-        emit_topk([&](int i) { return sm.key[i]; }, [&](int i) { return sm.idx[i]; }, cnt, kth, need, K, sm,
-                  io, so);
+        emit_topk([&](int i) { return sm.key[i]; }, [&](int i) { return sm.idx[i]; }, out_of, cnt, kth, need, K,
+                  sm, io, so);
     } else {
         // the guess failed: exact radix select over the whole row
         auto gkey = [&](int i) { return f32_order_key(row[i]); };
         radix_select(gkey, n, K, sm, &kth, &need);
-        emit_topk(gkey, [](int i) { return i; }, n, kth, need, K, sm, io, so);
+        emit_topk(gkey, [](int i) { return i; }, out_of, n, kth, need, K, sm, io, so);
     }
 }
 

@@ -106,7 +106,7 @@ class DecodeModel:
         self._w = (ctypes.c_void_p * self.S)(*[w.data_ptr() for w in self.W])
         self._wins = (csa2_window * self.L)(*[w.desc for w in self.windows])
         self.model = csa2_model(self.L, self.S, self._mode, self._src, self._idx_src, self._caches,
-                                self._w, self._wins, B, wl.H, wl.H_idx, wl.K, wl.scale)
+                                self._w, self._wins, B, wl.H, wl.H_idx, wl.K, wl.scale, wl.pool_blocks)
         self.ws = torch.empty(max(layer_step_workspace(self.model), 16), dtype=torch.uint8, device=device)
         # per-step buffers
         self.io = self.new_io()

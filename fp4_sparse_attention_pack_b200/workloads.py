@@ -106,6 +106,7 @@ class Workload:
     steps: int          # decode steps of the workload
     outliers: bool = False
     append: int = 0     # tokens appended per sequence before the decode steps
+    pool_blocks: int = 0  # > 0: hierarchical indexer, Reindex layers scan their source's pool
 
     @property
     def scale(self) -> float:
@@ -133,6 +134,11 @@ WORKLOADS = {
                 64, append=8192),
     # the pages' own schedule and ratios (8 scans per step, decoder source at ratio 1)
     5: Workload("cfg5_pages40_b16_128k", 5, 16, 131072, schedule_pages_40(), 64, 64, 512, 100),
+    # the hierarchical indexer on both schedules: pools of 2,048 blocks of 8 entries
+    6: Workload("cfg6_alternating40_b16_128k_pool2048", 2, 16, 131072, schedule_alternating_40(), 64, 64,
+                512, 100, pool_blocks=2048),
+    7: Workload("cfg7_pages40_b16_128k_pool2048", 5, 16, 131072, schedule_pages_40(), 64, 64, 512, 100,
+                pool_blocks=2048),
 }
 
 

@@ -192,6 +192,56 @@ int csa2_index_topk(const csa2_cache* cache, const uint16_t* q_idx, const float*
                     int K, int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
                     csa2_stream stream);
 
+/*
+ * Hierarchical sparse indexer ("DeepSeek-V4.1-Flash, expliqué pas à pas",
+ * CSA2 chapter, hierarchical indexer paragraph: the shallow indexer's result
+ * restricts what the deeper indexers may consider, and only the first Full
+ * layer keeps scanning the whole context; the video-summary page sizes the
+ * candidate pool at 2,048 blocks of 8 positions for a million tokens).  The
+ * page's step list did not survive; this library's reading:
+ *   - a block is 8 consecutive entries of a sequence (block j = entries
+ *     8j .. 8j + 7, the last block of a sequence possibly shorter);
+ *   - its score is the largest score of its entries under the Full layer's
+ *     indexer query (the csa2_index_topk score);
+ *   - the pool is the pool_blocks highest-scoring blocks (equal scores: lower
+ *     block first), written as block ids in increasing order, -1 padded when
+ *     the sequence has fewer blocks;
+ *   - a deeper layer scores only the entries of the pool's blocks (below
+ *     n_entries) and keeps the K best of them (equal scores: lower entry
+ *     first), written in increasing entry order, -1 padded.
+ * pool_blocks in 1..CSA2_MAX_POOL_BLOCKS.
+ */
+#define CSA2_MAX_POOL_BLOCKS 8192
+
+/* Workspace bytes of csa2_index_topk_pool and csa2_index_topk_in_pool. */
+size_t csa2_index_pool_workspace(int batch, int max_entries, int H_idx, int K, int pool_blocks);
+
+/*
+ * The Full layer's scan: exactly csa2_index_topk (idx_out, score_out), and in
+ * addition the pool of every sequence, pool_out int32 [batch][pool_blocks].
+ * ws must hold csa2_index_pool_workspace(batch, max_pages*64, H_idx, K,
+ * pool_blocks) bytes.  Errors as csa2_index_topk, plus INVALID_ARG for
+ * pool_blocks out of range or a NULL pool_out.
+ */
+int csa2_index_topk_pool(const csa2_cache* cache, const uint16_t* q_idx, const float* w, int H_idx,
+                         int K, int32_t* idx_out, float* score_out, int pool_blocks,
+                         int32_t* pool_out, void* ws, size_t ws_bytes, csa2_stream stream);
+
+/*
+ * A deeper layer's scan restricted to a pool: scores as csa2_index_topk but
+ * only for the entries of the blocks pool[b][0..pool_blocks), then the Top-K
+ * among them into idx_out [batch][K] (and score_out, nullable) as described
+ * above.  `pool` must be as csa2_index_topk_pool writes it (increasing valid
+ * block ids, then -1); block ids that are negative or at or beyond the
+ * sequence's blocks end the pool early.  A pool in another order gives a
+ * selection among its blocks' entries whose order and tie rule are not
+ * specified.  Same workspace and errors as csa2_index_topk_pool.
+ */
+int csa2_index_topk_in_pool(const csa2_cache* cache, const uint16_t* q_idx, const float* w,
+                            int H_idx, int K, const int32_t* pool, int pool_blocks,
+                            int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
+                            csa2_stream stream);
+
 /* Workspace bytes csa2_sparse_attn needs for these sizes. */
 size_t csa2_sparse_attn_workspace(int batch, int H, int K);
 
@@ -238,6 +288,11 @@ typedef struct {
     int32_t H_idx;                  /* indexer heads */
     int32_t K;                      /* Top-K */
     float scale;                    /* softmax scale (1/sqrt(512) in the tests) */
+    int32_t pool_blocks;            /* 0: every REINDEX layer scans its whole source;
+                                       1..CSA2_MAX_POOL_BLOCKS: hierarchical indexer, the
+                                       FULL layer of each source builds a pool of this many
+                                       blocks (csa2_index_topk_pool) and the REINDEX layers
+                                       of that source scan only it (csa2_index_topk_in_pool) */
 } csa2_model;
 
 /* Per-step inputs: host arrays of device pointers. */
@@ -264,7 +319,9 @@ size_t csa2_layer_step_workspace(const csa2_model* model);
  * One decode step of every layer.  Order: (1) each layer's window takes its
  * token; (2) each source takes its new token (an entry is written when a
  * ratio-2 pair completes); (3) every FULL/REINDEX layer scans its source with
- * its own indexer query and keeps the Top-K; (4) every layer attends: REUSE
+ * its own indexer query and keeps the Top-K (with pool_blocks > 0: the FULL
+ * layers first, each building its source's pool, then the REINDEX layers over
+ * the pools); (4) every layer attends: REUSE
  * layers over the indices of idx_src, SWA_ONLY layers over the window only.
  * Errors as the per-op calls; INVALID_ARG for an inconsistent mode table.
  */
@@ -307,6 +364,9 @@ int csa2_index_topk_noalloc(const csa2_cache* cache, const uint16_t* q_idx, cons
  *   [0] start            [1] after window append  [2] after cache write
  *   [3] after query quantisation                  [4] after the indexer scan
  *   [5] after Top-K      [6] after attention      [7] after the split combine
+ * With pool_blocks > 0, [3] and [4] follow the FULL layers' query
+ * quantisation and scan, and [5] follows everything else of the indexer: the
+ * FULL layers' Top-K, the pool build and the REINDEX layers' pool scans.
  * A phase with nothing to do gives two events with no work between them.
  */
 #define CSA2_STEP_EVENTS 8
@@ -356,7 +416,10 @@ int csa2_cache_import(const csa2_cache* cache, int seq, const void* image, int c
  * Number of kernel launches one csa2_layer_step(model, in, ...) call enqueues
  * on the current device (the measurement variant adds none): the window
  * append, two for the cache write when any source takes a token, three for the
- * indexer (query quantisation, scan, Top-K) when any layer scans, and one or two
+ * indexer (query quantisation, scan, Top-K) when any layer scans -- with
+ * pool_blocks > 0 plus two for the pool build (block maxima, their Top-K) and,
+ * when REINDEX layers exist, four for their pool scans (pool count, query
+ * quantisation, scan, Top-K) -- and one or two
  * for attention (a second one combines split tiles when there are fewer
  * (layer, sequence) pairs than SMs).  Returns a negative csa2_status when the
  * model table is invalid or `in` is NULL.  Enqueues nothing.

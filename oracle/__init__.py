@@ -205,14 +205,19 @@ def topk(scores, K) -> np.ndarray:
 POOL_BLOCK = 8
 
 
+def block_maxima(scores) -> np.ndarray:
+    """Score of every block: the largest score among its (up to 8) entries."""
+    scores = np.asarray(scores, np.float64)
+    if scores.size == 0:
+        return np.zeros(0, np.float64)
+    return np.maximum.reduceat(scores, np.arange(0, scores.size, POOL_BLOCK))
+
+
 def block_pool(scores, pool_blocks: int) -> np.ndarray:
     """Block ids of the pool, increasing, padded with -1 (int32[pool_blocks])."""
-    scores = np.asarray(scores, np.float64)
-    n = scores.size
-    if n == 0:
+    bmax = block_maxima(scores)
+    if bmax.size == 0:
         return np.full(pool_blocks, -1, np.int32)
-    starts = np.arange(0, n, POOL_BLOCK)
-    bmax = np.maximum.reduceat(scores, starts)
     return topk(bmax, pool_blocks)
 
 

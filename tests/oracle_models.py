@@ -38,7 +38,8 @@ def ref_model(wl, T=None):
     T = wl.T if T is None else T
     t = wl.table
     m = oracle.RefModel(t, wl.B, [wl.capacity_entries(s) for s in range(t.n_sources)],
-                        [W.w_idx(wl, s) for s in range(t.n_sources)], wl.H, wl.H_idx, wl.K, wl.scale)
+                        [W.w_idx(wl, s) for s in range(t.n_sources)], wl.H, wl.H_idx, wl.K, wl.scale,
+                        pool_blocks=wl.pool_blocks)
     for s in range(t.n_sources):
         m.caches[s] = ref_cache(wl, s, range(wl.B), T)
     for l in range(t.n_layers):

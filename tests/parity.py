@@ -4,6 +4,9 @@
 * Top-K: the GPU's index set equals the oracle's except for entries whose
   oracle score lies within TOPK_REL of the oracle's K-th score (their count is
   returned); indices distinct, within [0, n), increasing, padded with -1;
+* hierarchical indexer: the pool by the Top-K criterion over the oracle's block
+  maxima; a pool-restricted Top-K by the Top-K criterion over the oracle's
+  scores of the pool's entries;
 * attention: per (sequence, head) row, max_c |o - r| / max_c |r| <= ATTN_REL,
   the oracle evaluated on the GPU's own index set.
 """
@@ -41,3 +44,15 @@ def attn_rel_err(out: np.ndarray, ref: np.ndarray) -> float:
     r = np.asarray(ref, np.float64).reshape(-1, ref.shape[-1])
     den = np.maximum(np.abs(r).max(axis=1), 1e-30)
     return float((np.abs(o - r).max(axis=1) / den).max())
+
+
+def check_topk_in_pool(gpu_idx: np.ndarray, ref_scores: np.ndarray, cand: np.ndarray, K: int) -> int:
+    """Top-K criterion restricted to the candidate entries `cand` (increasing)."""
+    gpu_idx = np.asarray(gpu_idx, np.int64)
+    cand = np.asarray(cand, np.int64)
+    m = min(K, cand.size)
+    g = gpu_idx[:m]
+    pos = np.searchsorted(cand, g)
+    assert np.all(pos < cand.size) and np.array_equal(cand[np.minimum(pos, cand.size - 1)], g), \
+        "index outside the pool"
+    return check_topk(np.concatenate([pos, gpu_idx[m:]]), ref_scores[cand], K)

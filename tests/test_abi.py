@@ -117,3 +117,39 @@ def test_mode_table_validation(capi):
         sin, sout = capi.csa2_step_in(), capi.csa2_step_out()
         assert lib.csa2_layer_step(ctypes.byref(bad), ctypes.byref(sin), ctypes.byref(sout),
                                    ctypes.c_void_p(256), 1 << 30, None) == -1
+
+
+def test_pool_argument_checks(capi):
+    lib = capi.lib()
+    c = capi.csa2_cache(*([16] * 10), 1, 1, 1, 2)
+    p16 = ctypes.c_void_p(16)
+    assert capi.index_pool_workspace(2, 1024, 64, 512, 0) == 0
+    assert capi.index_pool_workspace(2, 1024, 64, 512, capi.MAX_POOL_BLOCKS + 1) == 0
+    # block maxima + pool counts on top of a scan whose rows hold max(entries, 8 * pool_blocks)
+    assert capi.index_pool_workspace(2, 1024, 64, 512, 2048) > capi.index_topk_workspace(2, 8 * 2048, 64, 512)
+    for pb in (0, capi.MAX_POOL_BLOCKS + 1):
+        assert lib.csa2_index_topk_pool(ctypes.byref(c), p16, p16, 4, 8, p16, None, pb, p16, p16, 1 << 30,
+                                        None) == -1
+        assert lib.csa2_index_topk_in_pool(ctypes.byref(c), p16, p16, 4, 8, p16, pb, p16, None, p16, 1 << 30,
+                                           None) == -1
+    assert lib.csa2_index_topk_pool(ctypes.byref(c), p16, p16, 4, 8, p16, None, 4, None, p16, 1 << 30,
+                                    None) == -1                                     # no pool_out
+    assert lib.csa2_index_topk_in_pool(ctypes.byref(c), p16, p16, 4, 8, ctypes.c_void_p(20), 4, p16, None,
+                                       p16, 1 << 30, None) == -2                    # unaligned pool
+    assert lib.csa2_index_topk_in_pool(ctypes.byref(c), p16, p16, 4, 8, p16, 4, p16, None, p16, 16,
+                                       None) == -6                                  # workspace too small
+
+
+def test_model_pool_blocks_range(capi):
+    from fp4_sparse_attention_pack_b200 import workloads as W
+    caches = (capi.csa2_cache * 1)(capi.csa2_cache(*([16] * 10), 1, 1, 1, 2))
+    wins = (capi.csa2_window * 3)(*[capi.csa2_window(16, 16, 1) for _ in range(3)])
+    ws = (ctypes.c_void_p * 1)(16)
+    keep = [(ctypes.c_int32 * 3)(W.FULL, W.REINDEX, W.REUSE), (ctypes.c_int32 * 3)(0, 0, 0),
+            (ctypes.c_int32 * 3)(0, 1, 1)]
+    sizes = {}
+    for pb in (0, 16, -1, capi.MAX_POOL_BLOCKS + 1):
+        m = capi.csa2_model(3, 1, keep[0], keep[1], keep[2], caches, ws, wins, 1, 4, 4, 8, 0.04, pb)
+        sizes[pb] = capi.layer_step_workspace(m)
+    assert sizes[-1] == 0 and sizes[capi.MAX_POOL_BLOCKS + 1] == 0
+    assert sizes[16] > sizes[0] > 0
