@@ -185,22 +185,21 @@ int csa2_index_topk_pool(const csa2_cache* cache, const uint16_t* q_idx, const f
     sb.p[0].idx_out = idx_out;
     sb.p[0].score_out = score_out;
     carve_scan_workspace(sb, wsp, cache->batch, pw.rows);
-    rc = cuda_status(launch_index_topk(sb, st));
+    rc = cuda_status(launch_quant_scan(sb, st));
     if (rc) return rc;
     float* bmax = reinterpret_cast<float*>(wsp + pw.scan);
     rc = cuda_status(launch_block_max(sb, bmax, pw.bstride, st));
     if (rc) return rc;
-    ScanBatch sp;
-    std::memset(&sp, 0, sizeof(sp));
-    sp.n = 1;
-    sp.H_idx = H_idx;
-    sp.K = pool_blocks;
-    sp.score_stride = pw.bstride;
-    sp.p[0].cache = sb.p[0].cache;
-    sp.p[0].scores = bmax;
-    sp.p[0].block_rows = 1;
-    sp.p[0].idx_out = pool_out;
-    return cuda_status(launch_topk(sp, st));
+    // one Top-K launch: the entries (K) and the block maxima (pool_blocks)
+    ScanProblem& B = sb.p[1];
+    B.cache = sb.p[0].cache;
+    B.scores = bmax;
+    B.row_stride = pw.bstride;
+    B.block_rows = 1;
+    B.K = pool_blocks;
+    B.idx_out = pool_out;
+    sb.n = 2;
+    return cuda_status(launch_topk(sb, st));
 }
 
 int csa2_index_topk_in_pool(const csa2_cache* cache, const uint16_t* q_idx, const float* w, int H_idx, int K,
@@ -490,10 +489,10 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
         P.score_out = nullptr;
     }
     carve_scan_workspace(sb, wsp, B, sw.rows);
-    if (sb.n > 0) {
+    if (sb.n > 0 && PB == 0) {
         rc = cuda_status(launch_index_topk(sb, st, ev ? ev + 3 : nullptr));
         if (rc) return rc;
-    } else if (ev) {
+    } else if (PB == 0 && ev) {
         for (int i = 3; i < 6; ++i) cudaEventRecord(ev[i], st);
     }
     if (PB > 0) {
@@ -501,26 +500,28 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
         int32_t* pools = reinterpret_cast<int32_t*>(region);
         float* bmax = reinterpret_cast<float*>(region + sw.pools);
         int32_t* pool_n = reinterpret_cast<int32_t*>(region + sw.pools + sw.bmax);
-        // the pool of each source: block maxima of its Full layer's scores, their Top-K
+        // the Full layers' scans, then the pool of each source: the block maxima of
+        // its Full layer's scores; one Top-K launch over the Full layers' entries
+        // (K) and their block maxima (pool_blocks)
+        rc = cuda_status(launch_quant_scan(sb, st, ev ? ev + 3 : nullptr));
+        if (rc) return rc;
         rc = cuda_status(launch_block_max(sb, bmax, sw.bstride, st));
         if (rc) return rc;
-        ScanBatch sp;
-        std::memset(&sp, 0, sizeof(sp));
-        sp.n = sb.n;
-        sp.H_idx = m->H_idx;
-        sp.K = PB;
-        sp.score_stride = sw.bstride;
+        const int n_full = sb.n;
         int li = 0;
         for (int l = 0; l < L; ++l) {
             if (m->mode[l] != CSA2_MODE_FULL) continue;
-            ScanProblem& P = sp.p[li];
+            ScanProblem& P = sb.p[n_full + li];
             P.cache = sb.p[li].cache;
             P.scores = bmax + (int64_t)li * B * sw.bstride;
+            P.row_stride = sw.bstride;
             P.block_rows = 1;
+            P.K = PB;
             P.idx_out = pools + (int64_t)m->src[l] * B * PB;
             ++li;
         }
-        rc = cuda_status(launch_topk(sp, st));
+        sb.n = 2 * n_full;
+        rc = cuda_status(launch_topk(sb, st));
         if (rc) return rc;
         // the Reindex layers over their sources' pools
         ScanBatch sr;
@@ -595,7 +596,7 @@ int csa2_layer_step_launches(const csa2_model* m, const csa2_step_in* in) {
         }
     if (n_scans(m) > 0) n += 3;  // query quantisation, scan, Top-K
     if (m->pool_blocks > 0) {
-        n += 2;                                        // block maxima, pool Top-K
+        n += 1;                                        // block maxima (the pool Top-K shares a launch)
         if (n_mode(m, CSA2_MODE_REINDEX) > 0) n += 4;  // pool count, quantisation, scan, Top-K
     }
     AttnBatch ab;

@@ -34,6 +34,8 @@ struct ScanProblem {
     int32_t* pool_n;        // [batch]
     int pool_blocks;
     int block_rows;         // the score row holds block maxima: ceil(n_entries / 8) of them
+    int K;                  // Top-K of this row (0: the batch's K)
+    int64_t row_stride;     // floats between sequences' score rows (0: the batch's score_stride)
 };
 
 constexpr int kMaxProblems = 64;
@@ -69,10 +71,12 @@ void carve_scan_workspace(ScanBatch& sb, uint8_t* ws, int batch, int max_entries
 // ev (nullable): events recorded after query quantisation, after the scan and
 // after Top-K (three cudaEvent_t).
 cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t* ev = nullptr);
+// The same without the Top-K (ev: two events).
+cudaError_t launch_quant_scan(const ScanBatch& sb, cudaStream_t st, cudaEvent_t* ev = nullptr);
 // Kernel launches one launch_index_topk(sb) call makes.
 int index_topk_launches(const ScanBatch& sb);
 
-// Top-K of every problem's score row (row_len positions), sb.K per row.
+// Top-K of every problem's score row (row_len positions), P.K (else sb.K) per row.
 cudaError_t launch_topk(const ScanBatch& sb, cudaStream_t st);
 
 // pool_n of every pool problem of sb: the valid prefix of its positions.

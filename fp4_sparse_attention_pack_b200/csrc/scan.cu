@@ -192,6 +192,14 @@ bool has_pool(const ScanBatch& sb) {
 int index_topk_launches(const ScanBatch& sb) { return 3 + (has_pool(sb) ? 1 : 0); }
 
 cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t* ev) {
+    cudaError_t e = launch_quant_scan(sb, st, ev);
+    if (e != cudaSuccess) return e;
+    e = launch_topk(sb, st);
+    if (e == cudaSuccess && ev) cudaEventRecord(ev[2], st);
+    return e;
+}
+
+cudaError_t launch_quant_scan(const ScanBatch& sb, cudaStream_t st, cudaEvent_t* ev) {
     const int batch = sb.p[0].cache.batch;
     if (has_pool(sb)) {
         cudaError_t e = launch_pool_count(sb, st);
@@ -220,9 +228,7 @@ cudaError_t launch_index_topk(const ScanBatch& sb, cudaStream_t st, cudaEvent_t*
         if (e != cudaSuccess) return e;
         if (ev) cudaEventRecord(ev[1], st);
     }
-    cudaError_t e = launch_topk(sb, st);
-    if (e == cudaSuccess && ev) cudaEventRecord(ev[2], st);
-    return e;
+    return cudaSuccess;
 }
 
 }  // namespace csa2

@@ -20,14 +20,20 @@
 //           64-byte swizzle) and bulk copies of their E8M0 scales into an
 //           8-stage ring; per work item the query tiles, scales and head
 //           weights of every problem of the subset (double-buffered).  Keys
-//           stream with an L2 evict-first policy.
-//   warp 1  MMA issuer: copies each item's query scales and each stage's key
-//           scales into TMEM (tcgen05.cp), then per tile issues one MMA pass per
-//           problem pair into one of two TMEM accumulators, committing each pass
-//           to its epilogue group and the stage back to the producer after the
-//           last pass.
-//   warps 2-17 epilogue, two groups of eight; group g drains the passes that
-//           landed in accumulator g.  Warp w of a group reads TMEM lane quadrant
+//           stream with an L2 evict-first policy.  Copies are issued by several
+//           lanes at once (a lane per page, per problem or per pool block):
+//           issuing them one by one from a single lane made this warp the
+//           bottleneck of the whole pipeline.
+//   warp 1  MMA issuer: per tile issues one MMA pass per
+//           problem pair into one of three TMEM accumulators (pass p into
+//           p % 3), committing each pass to its epilogue group.  Its only
+//           commits are those: the epilogue warp that sees a tile's last pass
+//           complete hands the key stage back to the producer, and the
+//           epilogue's arrivals after an item's last pass free the query
+//           buffer.  Three accumulators let the next pass run while both
+//           groups drain theirs.
+//   warps 2-17 epilogue, two groups of eight; group g drains the passes p with
+//           p % 2 == g.  Warp w of a group reads TMEM lane quadrant
 //           w % 4 and problem (w / 4) % 2 of the pass: tcgen05.ld of the 64 head
 //           columns of its entry, ReLU, weight, sum, one score store.
 //           A subset that scans a pool (hierarchical indexer) instead gathers
@@ -35,8 +41,11 @@
 //           own 512-byte slot, so the swizzled layout is that of a whole page.
 //   warp 18 scale warp: rearranges the E8M0 scales that landed in shared memory
 //           into the 32x128-bit layout tcgen05.cp reads (per item for the
-//           queries, per stage for the keys) and signals them ready, keeping
-//           the transposition and its proxy fence off the MMA issuer's path.
+//           queries, per stage for the keys), copies them into TMEM and commits
+//           the copies to the ready barriers the MMA issuer waits on, keeping
+//           the transposition, its proxy fence and the copies off the issuer's
+//           path (one tcgen05 instruction costs the issuing warp about a hundred
+//           cycles).
 // Every wait is bounded; a timeout sets CSA2_DEVERR_TIMEOUT in the problem's
 // status word and the CTA drains and exits.
 #include <cuda.h>
@@ -62,13 +71,14 @@ constexpr int kMaxPasses = kMaxSub / kPass;
 constexpr int kStages = 8;
 constexpr int kTile = 128;        // entries per MMA tile (MMA M)
 constexpr int kMaxChunk = 16;     // tiles per work item at most (32 pages: one per producer lane)
-constexpr int kGroups = 2;        // accumulators = epilogue groups
+constexpr int kGroups = 2;        // epilogue groups
+constexpr int kAcc = 3;           // TMEM accumulators: pass p lands in p % kAcc, group p % kGroups drains it
 constexpr int kEpiWarps = 8 * kGroups;
 constexpr int kSfWarp = 2 + kEpiWarps;
 constexpr int kThreads = 32 * (kSfWarp + 1);
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColAcc = 0;                            // kGroups x 128 accumulator columns
-constexpr uint32_t kColSfa = 128 * kGroups;                // kStages x 4 scale columns (keys)
+constexpr uint32_t kColAcc = 0;                            // kAcc x 128 accumulator columns
+constexpr uint32_t kColSfa = 128 * kAcc;                   // kStages x 4 scale columns (keys)
 constexpr uint32_t kColSfb = kColSfa + 4 * kStages;        // 2 x kMaxPasses x 4 (queries)
 static_assert(kColSfb + 2 * kMaxPasses * 4 <= kTmemCols, "TMEM columns");
 constexpr int kMaxSources = CSA2_MAX_SOURCES;
@@ -105,8 +115,8 @@ struct __align__(1024) Smem {
     int prow[kMaxChunk * 16];                // pool items: first physical key row of each slot
     uint64_t full[kStages], empty[kStages], sfa_ready[kStages];
     uint64_t bfull[2], bempty[2], sfb_ready[2];
-    uint64_t tfull[kGroups], tempty[kGroups];
-    uint64_t drained;
+    uint64_t tfull[kAcc], tempty[kAcc];
+    uint64_t drained, sdrained;
     uint32_t tmem_base;
     int abort;
 };
@@ -172,19 +182,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.empty[s], 1);  // the epilogue warp that sees the tile's last pass complete
             mbar_init(&sm.sfa_ready[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.bfull[i], 1);
-            mbar_init(&sm.bempty[i], 1 + kEpiWarps);
+            mbar_init(&sm.bempty[i], kEpiWarps);  // after the item's last pass: its MMAs are done
             mbar_init(&sm.sfb_ready[i], 1);
         }
-        for (int g = 0; g < kGroups; ++g) {
-            mbar_init(&sm.tfull[g], 1);
-            mbar_init(&sm.tempty[g], 8);  // the eight warps of epilogue group g
+        for (int a = 0; a < kAcc; ++a) {
+            mbar_init(&sm.tfull[a], 1);
+            mbar_init(&sm.tempty[a], 8);  // the eight warps of the group that drains it
         }
         mbar_init(&sm.drained, 1);
+        mbar_init(&sm.sdrained, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -226,15 +237,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane < S.n) sm.rows[bslot][lane] = sb.p[S.prob[lane]].scores + (int64_t)it.b * sb.score_stride;
                 __syncwarp();
                 mbar_expect_tx_w(&sm.bfull[bslot], S.n * (kHeads * 64 + kHeads * 4 + kHeads * 4));
-                for (int j = 0; j < S.n; ++j) {
-                    const int p = S.prob[j];
+                __syncwarp();
+                // lane j issues problem j's copies: one warp instruction per kind of copy
+                if (lane < S.n) {
+                    const int p = S.prob[lane];
                     const int64_t qrow = ((int64_t)p * batch + it.b) * kHeads;
-                    tma_load_2d_w(sm.b[bslot] + j * kHeads * 64, &mp.queries, 0, (int)qrow, &sm.bfull[bslot], pol_keep);
-                    bulk_load_w(sm.sfb_raw[bslot] + j * kHeads * 4, sb.qs + qrow * ISB, kHeads * 4, &sm.bfull[bslot],
-                                pol_keep);
-                    bulk_load_w(sm.w[bslot][j], sb.p[p].w + (int64_t)it.b * kHeads, kHeads * 4, &sm.bfull[bslot],
-                                pol_keep);
+                    tma_load_2d(sm.b[bslot] + lane * kHeads * 64, &mp.queries, 0, (int)qrow, &sm.bfull[bslot], pol_keep);
+                    bulk_load(sm.sfb_raw[bslot] + lane * kHeads * 4, sb.qs + qrow * ISB, kHeads * 4, &sm.bfull[bslot],
+                              pol_keep);
+                    bulk_load(sm.w[bslot][lane], sb.p[p].w + (int64_t)it.b * kHeads, kHeads * 4, &sm.bfull[bslot],
+                              pol_keep);
                 }
+                __syncwarp();
             }
             if (++bslot == 2) bslot = 0, bphase ^= 1;
             const CUtensorMap* kmap = &mp.keys[S.src];
@@ -292,16 +306,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_w(&sm.full[stage]);
                 } else {
                     mbar_expect_tx_w(&sm.full[stage], bytes);
-                    if (pg0 >= 0) {
-                        tma_load_2d_w(sm.a[stage], kmap, 0, pg0 * PAGE, &sm.full[stage], pol_stream);
-                        bulk_load_w(sm.sfa_raw[stage], c.idx_scales + (int64_t)pg0 * PAGE * ISB, PAGE * ISB,
-                                    &sm.full[stage], pol_stream);
+                    __syncwarp();
+                    // lanes 0, 1 load the two pages' key codes, lanes 2, 3 their scales
+                    const int h = lane & 1;
+                    const int pg = h ? pg1 : pg0;
+                    if (lane < 4 && pg >= 0) {
+                        if (lane < 2)
+                            tma_load_2d(sm.a[stage] + h * PAGE * ICB, kmap, 0, pg * PAGE, &sm.full[stage], pol_stream);
+                        else
+                            bulk_load(sm.sfa_raw[stage] + h * PAGE * ISB, c.idx_scales + (int64_t)pg * PAGE * ISB,
+                                      PAGE * ISB, &sm.full[stage], pol_stream);
                     }
-                    if (pg1 >= 0) {
-                        tma_load_2d_w(sm.a[stage] + PAGE * ICB, kmap, 0, pg1 * PAGE, &sm.full[stage], pol_stream);
-                        bulk_load_w(sm.sfa_raw[stage] + PAGE * ISB, c.idx_scales + (int64_t)pg1 * PAGE * ISB,
-                                    PAGE * ISB, &sm.full[stage], pol_stream);
-                    }
+                    __syncwarp();
                 }
                 issued |= 1u << stage;
                 issued_par = (issued_par & ~(1u << stage)) | (sphase << stage);
@@ -322,18 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const ScanSub& S = mp.sub[it.s];
             uint32_t* status = sb.p[S.prob[0]].cache.status;
             const int passes = (S.n + kPass - 1) / kPass;
+            // the query scales of the item are in TMEM once sfb_ready completes
             if (!mbar_wait_warp(&sm.sfb_ready[bslot], bphase)) { raise_abort(sm, status); break; }
-            // query scales of each pass -> TMEM (rows = the pass's 128 query rows)
-            tc_fence_after();
-            for (int k = 0; k < passes; ++k)
-                tc_cp_32x128b_x4_w(tbase + kColSfb + (bslot * kMaxPasses + k) * 4,
-                                   smem_desc(sm.sfb_tc[bslot][k], 16, 128, kLayoutNone));
             bool stop = false;
             for (int t = it.t0; t < it.t1; ++t) {
+                // ... and the stage's key scales once sfa_ready completes
                 if (!mbar_wait_warp(&sm.sfa_ready[stage], sphase)) { raise_abort(sm, status); stop = true; break; }
                 const uint32_t sfa = tbase + kColSfa + 4 * stage;
                 tc_fence_after();
-                tc_cp_32x128b_x4_w(sfa, smem_desc(sm.sfa_tc[stage], 16, 128, kLayoutNone));
                 const uint64_t adesc = smem_desc(sm.a[stage], 16, 512, kLayoutSw64);
                 for (int k = 0; k < passes; ++k) {
                     if (!mbar_wait_warp(&sm.tempty[acc], aphase ^ 1)) { raise_abort(sm, status); stop = true; break; }
@@ -346,13 +358,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_mma_mxf4_w(d, adesc, bdesc, idesc_mxf4(n_rows, 0, 0), sfa, sfb, 0u);
                     tc_mma_mxf4_w(d, adesc + 2, bdesc + 2, idesc_mxf4(n_rows, 2, 2), sfa, sfb, 1u);
                     tc_commit_w(&sm.tfull[acc]);
-                    if (++acc == kGroups) acc = 0, aphase ^= 1;
+                    if (++acc == kAcc) acc = 0, aphase ^= 1;
                 }
                 if (stop) break;
-                tc_commit_w(&sm.empty[stage]);
                 if (++stage == kStages) stage = 0, sphase ^= 1;
             }
-            tc_commit_w(&sm.bempty[bslot]);
             if (++bslot == 2) bslot = 0, bphase ^= 1;
             if (stop) break;
         }
@@ -366,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int jp = (ew >> 2) & 1;     // problem of the pass this warp reads
         const int quad = warp & 3;        // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;
-        uint32_t bslot = 0, bphase = 0, aphase = 0, pass_no = 0;
+        uint32_t bslot = 0, bphase = 0, pass_no = 0, stage = 0;
         for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
             Item it;
             if (!item_at(sb, mp, id, it)) continue;
@@ -375,15 +385,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t* status = sb.p[S.prob[0]].cache.status;
             if (!mbar_wait_warp(&sm.bfull[bslot], bphase)) { raise_abort(sm, status); break; }
             bool stop = false;
-            for (int t = it.t0; t < it.t1 && !stop; ++t) {
+            for (int t = it.t0; t < it.t1 && !stop; ++t, stage = stage + 1 == kStages ? 0 : stage + 1) {
                 for (int k = 0; k < passes; ++k, ++pass_no) {
                     if ((int)(pass_no % kGroups) != grp) continue;
-                    if (!mbar_wait_warp(&sm.tfull[grp], aphase)) { raise_abort(sm, status); stop = true; break; }
-                    aphase ^= 1;
+                    const int acc = (int)(pass_no % kAcc);
+                    if (!mbar_wait_warp(&sm.tfull[acc], (pass_no / kAcc) & 1u)) {
+                        raise_abort(sm, status);
+                        stop = true;
+                        break;
+                    }
+                    // the tile's last pass has completed, and every MMA before it:
+                    // its key stage goes back to the producer
+                    if (k == passes - 1 && (ew & 7) == 0 && lane == 0) mbar_arrive(&sm.empty[stage]);
                     tc_fence_after();
                     const int j = kPass * k + jp;
                     if (j < S.n) {
-                        const uint32_t taddr = tbase + ((uint32_t)(quad * 32) << 16) + kColAcc + 128 * grp + 64 * jp;
+                        const uint32_t taddr = tbase + ((uint32_t)(quad * 32) << 16) + kColAcc + 128 * acc + 64 * jp;
                         const float* w = sm.w[bslot][j];
                         float2 acc2[4];  // eight chains: heads h = 8i + c go to chain c
 #pragma unroll
@@ -395,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (half == 1) {
                                 tc_fence_before();
                                 __syncwarp();
-                                if (lane == 0) mbar_arrive(&sm.tempty[grp]);
+                                if (lane == 0) mbar_arrive(&sm.tempty[acc]);
                             }
 #pragma unroll
                             for (int h = 0; h < 32; h += 8) {
@@ -418,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm.tempty[grp]);
+                        if (lane == 0) mbar_arrive(&sm.tempty[acc]);
                     }
                 }
             }
@@ -437,10 +454,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t* status = sb.p[S.prob[0]].cache.status;
             const int passes = (S.n + kPass - 1) / kPass;
             if (!mbar_wait_warp(&sm.bfull[bslot], bphase)) { if (lane == 0) raise_abort(sm, status); break; }
+            // bfull implies the MMAs of the item two back, which read these TMEM
+            // columns, have completed (bempty follows its last pass's completion)
+            tc_fence_after();
             for (int k = 0; k < passes; ++k) scales_to_tc(sm.sfb_raw[bslot] + k * 512, sm.sfb_tc[bslot][k], lane);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.sfb_ready[bslot]);
+            for (int k = 0; k < passes; ++k)
+                tc_cp_32x128b_x4_w(tbase + kColSfb + (bslot * kMaxPasses + k) * 4,
+                                   smem_desc(sm.sfb_tc[bslot][k], 16, 128, kLayoutNone));
+            tc_commit_w(&sm.sfb_ready[bslot]);
             if (++bslot == 2) bslot = 0, bphase ^= 1;
             bool stop = false;
             for (int t = it.t0; t < it.t1; ++t) {
@@ -449,14 +472,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     stop = true;
                     break;
                 }
+                // full implies the MMAs that last read this stage's scale columns
+                // have completed (the stage's empty arrival follows them)
+                tc_fence_after();
                 scales_to_tc(sm.sfa_raw[stage], sm.sfa_tc[stage], lane);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.sfa_ready[stage]);
+                tc_cp_32x128b_x4_w(tbase + kColSfa + 4 * stage, smem_desc(sm.sfa_tc[stage], 16, 128, kLayoutNone));
+                tc_commit_w(&sm.sfa_ready[stage]);
                 if (++stage == kStages) stage = 0, sphase ^= 1;
             }
             if (stop) break;
         }
+        // every scale copy of this warp has completed before TMEM is freed
+        tc_commit_w(&sm.sdrained);
+        (void)mbar_wait_warp(&sm.sdrained, 0);
     }
 
     tc_fence_before();

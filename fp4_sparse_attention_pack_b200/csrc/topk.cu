@@ -169,9 +169,9 @@ __global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanB
     TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
     const ScanProblem& P = sb.p[blockIdx.y];
     const int b = blockIdx.x;
-    const int K = sb.K;
+    const int K = P.K > 0 ? P.K : sb.K;
     const int n = row_len(P, b);
-    const float* row = P.scores + (int64_t)b * sb.score_stride;
+    const float* row = P.scores + (int64_t)b * (P.row_stride > 0 ? P.row_stride : sb.score_stride);
     int32_t* io = P.idx_out + (int64_t)b * K;
     float* so = P.score_out ? P.score_out + (int64_t)b * K : nullptr;
     const int tid = threadIdx.x;
@@ -185,13 +185,15 @@ __global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanB
         return;
     }
 
-    // 1. threshold guess from strided samples (all scores qualify when they fit)
+    // 1. threshold guess from strided samples (all scores qualify when they fit):
+    // about 2K candidates, at most halfway from K to kCap
     uint32_t guess = 0;
-    if (n > kCap) {
+    if (n > kCap && K < kCap) {
         for (int i = tid; i < kSamples; i += kThreads)
             sm.key[i] = f32_order_key(row[(int64_t)i * n / kSamples]);
         __syncthreads();
-        const int rank = min(kSamples, (int)(((int64_t)2 * K * kSamples + n - 1) / n) + 16);
+        const int64_t target = min((int64_t)2 * K, (int64_t)(K + kCap) / 2);
+        const int rank = min(kSamples, (int)((target * kSamples + n - 1) / n) + 16);
         int unused;
         radix_select([&](int i) { return sm.key[i]; }, kSamples, rank, sm, &guess, &unused);
     }
@@ -200,8 +202,8 @@ __global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanB
     // thread takes a contiguous run of kRun scores, so a chunk of kThreads * kRun
     // scores costs four vector loads and one block scan per thread.
     int cnt = 0;
-    bool fits = true;
-    for (int base = 0; base < n; base += kThreads * kRun) {
+    bool fits = K < kCap;  // with K >= kCap the candidates never fit: straight to the exact select
+    for (int base = 0; fits && base < n; base += kThreads * kRun) {
         const int i0 = base + tid * kRun;
         uint32_t kk[kRun];
         if (i0 + kRun <= n) {

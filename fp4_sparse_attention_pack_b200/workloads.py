@@ -149,6 +149,9 @@ PROFILE_WORKLOADS = {
     "scan32": Workload("scan32_1layer_b32_128k", 5, 32, 131072, single_full(), 64, 64, 512, 4),
     # the 40-layer step at batch 4: 160 attention units (about one wave), 410 MB of keys per step
     "step_b4": Workload("step_b4_40layer_128k", 6, 4, 131072, schedule_alternating_40(), 64, 64, 512, 4),
+    # the same step with the hierarchical indexer (pools of 2,048 blocks)
+    "step_b4_pool": Workload("step_b4_pool2048_40layer_128k", 6, 4, 131072, schedule_alternating_40(), 64, 64,
+                             512, 4, pool_blocks=2048),
 }
 
 

@@ -417,7 +417,8 @@ int csa2_cache_import(const csa2_cache* cache, int seq, const void* image, int c
  * on the current device (the measurement variant adds none): the window
  * append, two for the cache write when any source takes a token, three for the
  * indexer (query quantisation, scan, Top-K) when any layer scans -- with
- * pool_blocks > 0 plus two for the pool build (block maxima, their Top-K) and,
+ * pool_blocks > 0 plus one for the block maxima (their Top-K shares the FULL
+ * layers' Top-K launch) and,
  * when REINDEX layers exist, four for their pool scans (pool count, query
  * quantisation, scan, Top-K) -- and one or two
  * for attention (a second one combines split tiles when there are fewer
