@@ -146,6 +146,7 @@ def workload_config(wl, world):
            "cache_format": "E2M1+E4M3/16 main, MXFP4 indexer keys"}
     if wl.pool_blocks > 0:
         cfg["pool_blocks"] = wl.pool_blocks
+    cfg["window"] = "fp8 e4m3 (512 B a token)" if wl.win_fp8 else "bf16 (1,024 B a token)"
     return cfg
 
 
@@ -157,8 +158,8 @@ def kernel_bytes(wl, n_entries):
                   head weights, one fp32 score per (scan, entry) written;
       topk        the scores read, K indices written per (scan, sequence);
       attention   per (layer, sequence) the K selected entries (256 code + 32
-                  scale bytes) and their indices, the 128-token bf16 window, the
-                  bf16 query, the fp32 output;
+                  scale bytes) and their indices, the 128-token window (bf16, or
+                  one E4M3 byte a channel), the bf16 query, the fp32 output;
       step        all kernels, plus the cache write of the new tokens.
     With pools (hierarchical indexer) index_scan covers the Full layers only,
     and topk the rest of the indexer phase: the Full layers' Top-K, the block
@@ -190,8 +191,9 @@ def kernel_bytes(wl, n_entries):
         scan = (sum(n_src[s] * 68 for s in scanned) + len(scans) * qbytes + score_bytes)
         topk = score_bytes + len(scans) * B * K * 4
     attn = 0
+    win_b = 1 if wl.win_fp8 else 2  # bytes a window channel
     for m in t.mode:
-        attn += B * (WIN * 512 * 2 + H * 512 * 2 + H * 512 * 4)
+        attn += B * (WIN * 512 * win_b + H * 512 * 2 + H * 512 * 4)
         if m != 0:
             attn += B * K * (288 + 4)
     cache_write = t.n_sources * B * (512 * 2 + 4 + 288 + 68)

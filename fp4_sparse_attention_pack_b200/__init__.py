@@ -14,7 +14,8 @@ from ._build import LIB
 
 __all__ = ["Csa2Error", "lib", "csa2_cache", "csa2_window", "csa2_model", "csa2_step_in",
            "csa2_step_out", "pack_cache", "index_topk", "index_topk_workspace", "index_pool_workspace",
-           "index_topk_pool", "index_topk_in_pool", "POOL_BLOCK", "MAX_POOL_BLOCKS", "sparse_attn",
+           "index_topk_pool", "index_topk_in_pool", "POOL_BLOCK", "MAX_POOL_BLOCKS", "WIN_BF16", "WIN_FP8",
+           "sparse_attn",
            "sparse_attn_workspace", "window_append", "layer_step", "layer_step_workspace", "layer_step_launches", "seq_image_bytes", "cache_export",
            "cache_import",
            "SWA_ONLY", "FULL", "REINDEX", "REUSE", "DTYPE_BF16", "DTYPE_F32"]
@@ -22,6 +23,7 @@ __all__ = ["Csa2Error", "lib", "csa2_cache", "csa2_window", "csa2_model", "csa2_
 SWA_ONLY, FULL, REINDEX, REUSE = 0, 1, 2, 3
 DTYPE_BF16, DTYPE_F32 = 0, 1
 POOL_BLOCK, MAX_POOL_BLOCKS = 8, 8192
+WIN_BF16, WIN_FP8 = 0, 1
 DEVERR_CAPACITY, DEVERR_PAGE, DEVERR_COUNT, DEVERR_TIMEOUT, DEVERR_IMAGE = 1, 2, 4, 8, 16
 
 _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
@@ -41,7 +43,7 @@ class csa2_cache(ctypes.Structure):
 
 
 class csa2_window(ctypes.Structure):
-    _fields_ = [("tokens", _vp), ("count", _vp), ("batch", _i32)]
+    _fields_ = [("tokens", _vp), ("count", _vp), ("batch", _i32), ("dtype", _i32)]
 
 
 class csa2_model(ctypes.Structure):

@@ -36,6 +36,7 @@ int check_cache(const csa2_cache* c) {
 
 int check_window(const csa2_window* w, int batch) {
     if (!w || !w->tokens || !w->count || w->batch != batch) return CSA2_ERR_INVALID_ARG;
+    if (w->dtype != CSA2_WIN_BF16 && w->dtype != CSA2_WIN_FP8) return CSA2_ERR_INVALID_ARG;
     if (!a16(w->tokens) || !a16(w->count)) return CSA2_ERR_ALIGN;
     return CSA2_OK;
 }
@@ -268,6 +269,7 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const in
     P.q = q;
     P.idx = idx;
     P.win = win->tokens;
+    P.win_fp8 = win->dtype == CSA2_WIN_FP8;
     P.win_count = win->count;
     P.out = out;
     P.K = K;
@@ -285,6 +287,7 @@ int csa2_window_append(const csa2_window* win, const uint16_t* tok, csa2_stream 
     wa.n = 1;
     wa.batch = win->batch;
     wa.tokens[0] = win->tokens;
+    wa.fp8[0] = win->dtype == CSA2_WIN_FP8;
     wa.count[0] = win->count;
     wa.tok[0] = tok;
     return cuda_status(launch_window_append(wa, (cudaStream_t)stream));
@@ -445,6 +448,7 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
     wa.batch = B;
     for (int l = 0; l < L; ++l) {
         wa.tokens[l] = m->windows[l].tokens;
+        wa.fp8[l] = m->windows[l].dtype == CSA2_WIN_FP8;
         wa.count[l] = m->windows[l].count;
         wa.tok[l] = in->win_tok[l];
     }
@@ -559,6 +563,7 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
         AttnProblem& P = ab.p[l];
         P.q = in->q[l];
         P.win = m->windows[l].tokens;
+        P.win_fp8 = m->windows[l].dtype == CSA2_WIN_FP8;
         P.win_count = m->windows[l].count;
         P.out = out->out[l];
         P.idx = m->mode[l] == CSA2_MODE_SWA_ONLY ? nullptr : out->idx[m->idx_src[l]];

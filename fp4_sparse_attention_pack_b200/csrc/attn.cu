@@ -63,9 +63,24 @@ __global__ void __launch_bounds__(kThreads) k_attn_split(AttnBatch ab) {
                     }
                 }
             }
+        } else if (pos - K < wlen && P.win_fp8) {
+            ok = 1;
+            const uint8_t* src = static_cast<const uint8_t*>(P.win) + ((int64_t)b * WIN + (pos - K)) * D + 16 * lane;
+            const uint4 u = *reinterpret_cast<const uint4*>(src);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                for (int hlf = 0; hlf < 2; ++hlf) {
+                    const uint32_t hb = e4m3x2_to_h2((w[k] >> (16 * hlf)) & 0xFFFFu);
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hb));
+                    row[16 * lane + 4 * k + 2 * hlf] = f.x;
+                    row[16 * lane + 4 * k + 2 * hlf + 1] = f.y;
+                }
+            }
         } else if (pos - K < wlen) {
             ok = 1;
-            const uint16_t* src = P.win + ((int64_t)b * WIN + (pos - K)) * D + 16 * lane;
+            const uint16_t* src = static_cast<const uint16_t*>(P.win) + ((int64_t)b * WIN + (pos - K)) * D + 16 * lane;
             const uint4 u0 = *reinterpret_cast<const uint4*>(src);
             const uint4 u1 = *reinterpret_cast<const uint4*>(src + 8);
             const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
@@ -163,14 +178,39 @@ __global__ void k_attn_combine(AttnBatch ab) {
     for (int i = 0; i < 4; ++i) o[threadIdx.x + 128 * i] = acc[i] * inv;
 }
 
+// Eight bf16 channels (one 16-byte chunk) -> eight E4M3 codes: nearest finite
+// value, ties to even, saturating at +-448 (cvt ... satfinite).
+__device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 u) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        uint16_t lo, hi;
+        // cvt packs its first source operand into the upper byte
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(lo)
+            : "f"(__uint_as_float(w[2 * k] & 0xFFFF0000u)), "f"(__uint_as_float(w[2 * k] << 16)));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(hi)
+            : "f"(__uint_as_float(w[2 * k + 1] & 0xFFFF0000u)), "f"(__uint_as_float(w[2 * k + 1] << 16)));
+        o[k] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    return make_uint2(o[0], o[1]);
+}
+
 __global__ void k_window_append(WinAppend wa) {
     const int l = blockIdx.y, b = blockIdx.x;
     const int cnt = wa.count[l][b];
     __syncthreads();
     const int slot = ((cnt % WIN) + WIN) % WIN;
     const uint4* src = reinterpret_cast<const uint4*>(wa.tok[l] + (int64_t)b * D);
-    uint4* dst = reinterpret_cast<uint4*>(wa.tokens[l] + ((int64_t)b * WIN + slot) * D);
-    for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = src[i];
+    if (wa.fp8[l]) {
+        uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(wa.tokens[l]) + ((int64_t)b * WIN + slot) * D);
+        for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = bf16x8_to_e4m3x8(src[i]);
+    } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(wa.tokens[l]) + ((int64_t)b * WIN + slot) * D);
+        for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = src[i];
+    }
     if (threadIdx.x == 0) wa.count[l][b] = cnt + 1;
 }
 

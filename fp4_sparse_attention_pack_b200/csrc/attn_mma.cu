@@ -3,7 +3,8 @@
 //
 // Per (problem, sequence) the items are the K selected entries (dequantised
 // from E2M1 x E4M3: exact in fp16) and the valid window tokens (bf16 -> fp16,
-// exact for |x| in fp16's normal range); the latent item is key and value.
+// exact for |x| in fp16's normal range; E4M3 -> fp16, always exact, for an FP8
+// window); the latent item is key and value.
 // Items go through 128-item tiles with an online softmax:
 //
 //   S^T[128 items x 64 heads] = Items . Q^T            (M = 128, N = 64, K = 512)
@@ -20,7 +21,8 @@
 // Gather: the unit's selected entries and window are prefetched into L2 first;
 // window rows arrive by TMA (a 3-D tensor map per window, 128-byte swizzle, one
 // box per slab, so they land directly in the slab layout and are converted
-// bf16 -> fp16 in place); cache entries are loaded with 16-byte loads into
+// bf16 -> fp16 in place); FP8 window rows (64 bytes a slab) are loaded with
+// 16-byte loads when their tile is built; cache entries are loaded with 16-byte loads into
 // registers one tile ahead (warp w: slab w % 8, rows 64 (w / 8) .. + 63, two rows
 // per lane) and dequantised into the swizzled slab; a slab is rewritten as soon
 // as the previous tile's O block that reads it has completed (the O MMAs commit
@@ -204,8 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        if (tid == 0 && t_end * kT > K && wlen > 0)
-            bulk_prefetch_l2(P.win + (int64_t)b * WIN * D, (uint32_t)wlen * D * 2);
+        if (tid == 0 && t_end * kT > K && wlen > 0) {
+            const int tb = P.win_fp8 ? 1 : 2;  // bytes a channel
+            bulk_prefetch_l2(static_cast<const uint8_t*>(P.win) + (int64_t)b * WIN * D * tb, (uint32_t)wlen * D * tb);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -238,7 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else if (pos - K < wlen) {
-                kind = 2;
+                kind = P.win_fp8 ? 3 : 2;
+                row = (int64_t)b * WIN + (pos - K);
             }
             sm.kind[buf][tid] = kind;
             sm.src_row[buf][tid] = row;
@@ -308,6 +313,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int kind = sm.kind[buf][r];
                 if (kind == 2) {
                     bf16_row_to_f16(sm.items[j], r);
+                } else if (kind == 3) {
+                    // FP8 window token: the slab's 64 E4M3 codes -> fp16 (exact)
+                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(P.win) +
+                                                                      sm.src_row[buf][r] * D + 64 * j);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const uint4 u = __ldg(src + q4);
+                        const uint32_t cw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {  // 16-byte chunk 2 q4 + cc: channels 8 (2 q4 + cc) ..
+                            uint4 o;
+                            o.x = e4m3x2_to_h2(cw[2 * cc] & 0xFFFFu);
+                            o.y = e4m3x2_to_h2(cw[2 * cc] >> 16);
+                            o.z = e4m3x2_to_h2(cw[2 * cc + 1] & 0xFFFFu);
+                            o.w = e4m3x2_to_h2(cw[2 * cc + 1] >> 16);
+                            *reinterpret_cast<uint4*>(sm.items[j] + sw128(r, 2 * q4 + cc)) = o;
+                        }
+                    }
                 } else if (kind == 0) {
                     zero_row(sm.items[j], r);
                 } else {
@@ -609,8 +632,8 @@ cudaError_t launch_attn_mma(const AttnBatch& ab_in, cudaStream_t st, cudaEvent_t
     AttnBatch ab = ab_in;
     AttnMaps maps;  // kernel parameter (copied at launch)
     std::memset(&maps, 0, sizeof(maps));
-    for (int i = 0; i < ab.n; ++i)
-        if (!make_window_map(&maps.win[i], ab.p[i].win, ab.batch)) return cudaErrorInvalidValue;
+    for (int i = 0; i < ab.n; ++i)  // FP8 windows are gathered, not loaded by TMA
+        if (!ab.p[i].win_fp8 && !make_window_map(&maps.win[i], ab.p[i].win, ab.batch)) return cudaErrorInvalidValue;
     const int splits = attn_mma_splits(ab.n, ab.batch, ab.Kmax);
     const int tiles = (ab.Kmax + WIN + kT - 1) / kT;
     const int tps = (tiles + splits - 1) / splits;

@@ -8,6 +8,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -56,6 +57,14 @@ __device__ __forceinline__ float e2m1_decode(uint32_t code) {
 // Nearest-even E4M3 with saturation to +-448 (hardware cvt, sm_89+).
 __device__ __forceinline__ uint32_t e4m3_encode(float v) {
     return (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Two E4M3 codes (low byte = first channel) -> fp16x2 bits (exact: every E4M3
+// value is an fp16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
+    uint32_t out;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(out) : "r"(two));
+    return out;
 }
 
 // Exact fp32 value of a non-negative E4M3 code (the scales are never negative).

@@ -95,8 +95,9 @@ struct AttnProblem {
     CacheView cache;          // valid when K > 0
     const uint16_t* q;        // bf16 [batch][H][512]
     const int32_t* idx;       // [batch][K] or null (K == 0)
-    const uint16_t* win;      // bf16 [batch][128][512]
+    const void* win;          // bf16 or E4M3 (win_fp8) [batch][128][512]
     const int32_t* win_count; // [batch]
+    int win_fp8;
     float* out;               // fp32 [batch][H][512]
     int K;                    // 0 for window-only layers
 };
@@ -120,9 +121,10 @@ cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t
 
 // ---- window
 struct WinAppend {
-    uint16_t* tokens[kMaxProblems];
+    void* tokens[kMaxProblems];      // bf16 or E4M3 (fp8[l]) rings
     int32_t* count[kMaxProblems];
     const uint16_t* tok[kMaxProblems];
+    int fp8[kMaxProblems];
     int n;
     int batch;
 };

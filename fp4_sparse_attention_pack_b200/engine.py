@@ -12,8 +12,8 @@ import ctypes
 import numpy as np
 import torch
 
-from . import (csa2_cache, csa2_model, csa2_step_in, csa2_step_out, csa2_window, layer_step,
-               layer_step_workspace, pack_cache, synth, workloads as W)
+from . import (WIN_BF16, WIN_FP8, csa2_cache, csa2_model, csa2_step_in, csa2_step_out, csa2_window,
+               layer_step, layer_step_workspace, pack_cache, synth, window_append, workloads as W)
 
 D, D_IDX, WIN, PAGE = 512, 128, 128, 64
 
@@ -68,10 +68,14 @@ class DeviceCache:
 
 
 class DeviceWindow:
-    def __init__(self, B: int, device="cuda"):
-        self.tokens = torch.zeros(B, WIN, D, dtype=torch.bfloat16, device=device)
+    """One layer's SWA ring: bf16 tokens, or E4M3 codes when fp8."""
+
+    def __init__(self, B: int, device="cuda", fp8: bool = False):
+        self.fp8 = fp8
+        dt = torch.uint8 if fp8 else torch.bfloat16
+        self.tokens = torch.zeros(B, WIN, D, dtype=dt, device=device)
         self.count = torch.zeros(B, dtype=torch.int32, device=device)
-        self.desc = csa2_window(self.tokens.data_ptr(), self.count.data_ptr(), B)
+        self.desc = csa2_window(self.tokens.data_ptr(), self.count.data_ptr(), B, WIN_FP8 if fp8 else WIN_BF16)
 
 
 def _ptr_array(tensors):
@@ -95,7 +99,7 @@ class DecodeModel:
             max_pages = (cap_tokens // t.ratios[s] + PAGE - 1) // PAGE
             self.caches.append(DeviceCache(B, max_pages, t.ratios[s], device,
                                            None if page_seed is None else page_seed + s))
-        self.windows = [DeviceWindow(B, device) for _ in range(self.L)]
+        self.windows = [DeviceWindow(B, device, wl.win_fp8) for _ in range(self.L)]
         self.W = [torch.from_numpy(W.w_idx(wl, s)).to(device) for s in range(self.S)]
         self.chan = [torch.from_numpy(W.chan_scale(wl, s)).to(device) for s in range(self.S)]
         # model table (host arrays kept alive with the struct)
@@ -200,9 +204,16 @@ class DecodeModel:
         k = synth.key(wl.seed, synth.TID_WIN, l)
         tmp = torch.empty(B, n, D, dtype=torch.bfloat16, device=self.dev)
         synth.dev_normal_bf16_rows(tmp, k, p0 * D, synth.TSTRIDE * D, B, n * D)
+        win = self.windows[l]
+        if win.fp8:
+            # the library encodes: replay the tokens through the window append
+            win.count.fill_(p0)
+            for i in range(n):
+                window_append(win.desc, tmp[:, i].contiguous())
+            return
         slots = (torch.arange(p0, T, device=self.dev) % WIN)
-        self.windows[l].tokens[:, slots] = tmp
-        self.windows[l].count.fill_(T)
+        win.tokens[:, slots] = tmp
+        win.count.fill_(T)
 
     def gen_step_inputs(self, st: int):
         """Seeded inputs of decode step st (token position T + st) on the device."""

@@ -107,6 +107,7 @@ class Workload:
     outliers: bool = False
     append: int = 0     # tokens appended per sequence before the decode steps
     pool_blocks: int = 0  # > 0: hierarchical indexer, Reindex layers scan their source's pool
+    win_fp8: bool = False  # SWA windows kept as E4M3 codes instead of bf16
 
     @property
     def scale(self) -> float:
@@ -139,6 +140,9 @@ WORKLOADS = {
                 512, 100, pool_blocks=2048),
     7: Workload("cfg7_pages40_b16_128k_pool2048", 5, 16, 131072, schedule_pages_40(), 64, 64, 512, 100,
                 pool_blocks=2048),
+    # the 40-layer step with the SWA windows in FP8 (E4M3, 512 B a token)
+    8: Workload("cfg8_40layer_b16_128k_fp8win", 2, 16, 131072, schedule_alternating_40(), 64, 64, 512, 100,
+                win_fp8=True),
 }
 
 

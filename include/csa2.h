@@ -130,15 +130,27 @@ typedef struct {
 
 /*
  * One layer's SWA window for `batch` sequences ("une branche locale SWA qui
- * maintient le KV SWA des 128 derniers tokens"): a ring of 128 bf16 tokens of
- * 512 channels.  Token number t (0-based, counted per sequence) sits in slot
+ * maintient le KV SWA des 128 derniers tokens"): a ring of 128 tokens of 512
+ * channels.  Token number t (0-based, counted per sequence) sits in slot
  * t % 128; count[b] tokens were appended, the first min(count[b], 128) slots
  * are valid.  Attention is order-free, so the ring needs no rotation.
+ *
+ * dtype CSA2_WIN_BF16: tokens are bf16 [batch][128][512] (1,024 B a token).
+ * dtype CSA2_WIN_FP8 ("Le cache KV en FP4": the SWA KV stays in FP8, being more
+ * sensitive to quantisation): tokens are E4M3 codes uint8 [batch][128][512]
+ * (512 B a token, half the bf16 ring).  The pages give no scale for it, and
+ * the FP8 main entry of V4 they cite is 512 bytes for 512 channels, so none is
+ * kept: each channel is the nearest finite E4M3 value of the bf16 input (ties
+ * to the even code, saturating at +-448, a negative value rounding to zero
+ * keeps its sign).  E4M3 values are exact in fp16 and fp32.
  */
+#define CSA2_WIN_BF16 0
+#define CSA2_WIN_FP8 1
 typedef struct {
-    uint16_t* tokens; /* bf16 [batch][128][512] */
+    void* tokens;     /* bf16 or E4M3 [batch][128][512], per dtype */
     int32_t* count;   /* [batch] */
     int32_t batch;
+    int32_t dtype;    /* CSA2_WIN_BF16 or CSA2_WIN_FP8 */
 } csa2_window;
 
 /* Library version, (major << 16) | minor. */
@@ -261,7 +273,8 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const in
                      const csa2_window* win, float scale, float* out, void* ws, size_t ws_bytes,
                      csa2_stream stream);
 
-/* SWA ring write: tok bf16 [batch][512] goes to slot count % 128; count += 1. */
+/* SWA ring write: tok bf16 [batch][512] goes to slot count % 128 (as E4M3 codes
+ * for an FP8 window); count += 1.  INVALID_ARG for an unknown dtype. */
 int csa2_window_append(const csa2_window* win, const uint16_t* tok, csa2_stream stream);
 
 /*

@@ -55,6 +55,7 @@ def lib():
         for name, res, args in [
             ("ref_e2m1_value", cd, [cu]), ("ref_e4m3_value", cd, [cu]), ("ref_e8m0_value", cd, [cu]),
             ("ref_e2m1_encode", cu, [cf]), ("ref_e4m3_encode", cu, [cf]),
+            ("ref_window_fp8", None, [vp, ci, vp]),
             ("ref_mx_shared_exp", ci, [cf]), ("ref_spec_exp", cf, [cf]),
             ("ref_compress_pair", None, [vp, cf, vp, cf, vp]),
             ("ref_pack_main", None, [vp, vp, vp]), ("ref_dequant_main", None, [vp, vp, vp]),
@@ -107,6 +108,26 @@ def e2m1_encode(v: float) -> int:
 
 def e4m3_encode(v: float) -> int:
     return lib().ref_e4m3_encode(float(np.float32(v)))
+
+
+def window_fp8(tok_bf16) -> np.ndarray:
+    """E4M3 codes of bf16 window tokens, one per channel, same shape (the FP8
+    SWA window: "Le cache KV en FP4", the SWA KV stays in FP8)."""
+    x = np.ascontiguousarray(bf16_to_f32(tok_bf16), np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().ref_window_fp8(_p(x), x.size, _p(out))
+    return out
+
+
+_E4M3_VALUES = None
+
+
+def e4m3_values(codes) -> np.ndarray:
+    """fp32 values of E4M3 codes (each exact in fp32), from ref_e4m3_value."""
+    global _E4M3_VALUES
+    if _E4M3_VALUES is None:
+        _E4M3_VALUES = np.array([e4m3_value(c) for c in range(256)], np.float32)
+    return _E4M3_VALUES[np.asarray(codes, np.uint8)]
 
 
 def mx_shared_exp(amax: float) -> int:
@@ -249,6 +270,14 @@ def attention_items(mc, ms, n_entries, idx, win_bf16, win_len) -> np.ndarray:
     return items[:m]
 
 
+def attention_items_fp8(mc, ms, n_entries, idx, win_codes, win_len) -> np.ndarray:
+    """attention_items for an FP8 window: the selected entries, then the E4M3
+    values of the first win_len window slots."""
+    ents = attention_items(mc, ms, n_entries, idx, np.zeros((1, D), np.uint16), 0)
+    w = e4m3_values(np.asarray(win_codes, np.uint8).reshape(-1, D)[:win_len])
+    return np.concatenate([ents, w.astype(np.float32)])
+
+
 def attention(q_bf16, items, scale) -> np.ndarray:
     q = np.ascontiguousarray(bf16_to_f32(q_bf16).reshape(-1, D))
     items = np.ascontiguousarray(items, np.float32)
@@ -297,13 +326,15 @@ class RefModel:
     """All layers of one decode model: per-source caches and per-layer windows."""
 
     def __init__(self, table, B: int, caps, Ws, H: int, H_idx: int, K: int, scale: float,
-                 pool_blocks: int = 0):
+                 pool_blocks: int = 0, win_fp8: bool = False):
         self.t = table
         self.B, self.H, self.H_idx, self.K, self.scale = B, H, H_idx, K, scale
         self.pool_blocks = pool_blocks  # > 0: Reindex layers search the Full layer's pool
+        self.win_fp8 = win_fp8          # windows keep E4M3 codes (win8) instead of bf16
         self.caches = [RefCache(B, caps[s], table.ratios[s], Ws[s]) for s in range(table.n_sources)]
         L = table.n_layers
         self.win = np.zeros((L, B, WIN, D), np.uint16)
+        self.win8 = np.zeros((L, B, WIN, D), np.uint8) if win_fp8 else None
         self.win_count = np.zeros((L, B), np.int64)
         for l in range(L):
             m = table.mode[l]
@@ -316,6 +347,8 @@ class RefModel:
     def window_append(self, l: int, b: int, tok_bf16):
         slot = int(self.win_count[l, b] % WIN)
         self.win[l, b, slot] = np.asarray(tok_bf16, np.uint16).reshape(D)
+        if self.win_fp8:
+            self.win8[l, b, slot] = window_fp8(self.win[l, b, slot])
         self.win_count[l, b] += 1
 
     def win_len(self, l: int, b: int) -> int:
@@ -323,12 +356,14 @@ class RefModel:
 
     def layer_attention(self, l: int, b: int, q_bf16, idx) -> np.ndarray:
         wl = self.win_len(l, b)
+        gather = attention_items_fp8 if self.win_fp8 else attention_items
+        win = self.win8[l, b] if self.win_fp8 else self.win[l, b]
         if self.t.mode[l] == SWA_ONLY or idx is None:
-            items = attention_items(np.zeros((1, 256), np.uint8), np.zeros((1, 32), np.uint8), 0,
-                                    np.zeros(0, np.int32), self.win[l, b], wl)
+            items = gather(np.zeros((1, 256), np.uint8), np.zeros((1, 32), np.uint8), 0,
+                           np.zeros(0, np.int32), win, wl)
         else:
             c = self.caches[self.t.src[l]]
-            items = attention_items(c.mc[b], c.ms[b], int(c.n[b]), idx, self.win[l, b], wl)
+            items = gather(c.mc[b], c.ms[b], int(c.n[b]), idx, win, wl)
         return attention(q_bf16, items, self.scale)
 
     def step(self, x_new, g_new, q, qidx, wh, wtok, want=None):

@@ -82,6 +82,15 @@ unsigned ref_e4m3_encode(float v) {
     return sign | best;
 }
 
+/* SWA window in FP8 ("Le cache KV en FP4": the SWA KV stays in FP8, being more
+ * sensitive to quantisation).  The pages give no scale, and the FP8 main entry
+ * of V4 they cite takes 512 bytes for 512 channels, so none: one E4M3 code per
+ * channel, the nearest finite E4M3 value of the input (ref_e4m3_encode: ties to
+ * the even code, saturating at 448, sign kept). */
+void ref_window_fp8(const float* x, int n, uint8_t* codes) {
+    for (int i = 0; i < n; ++i) codes[i] = (uint8_t)ref_e4m3_encode(x[i]);
+}
+
 /* OCP MX v1.0 shared scale for FP4 elements: X = floor(log2(amax)) - emax_elem,
  * emax_elem = 2 (6 = 1.5 * 2^2), clamped to the E8M0 range [-127, 127]. */
 int ref_mx_shared_exp(float amax) {

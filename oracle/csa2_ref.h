@@ -32,6 +32,7 @@ double ref_e4m3_value(unsigned code);
 double ref_e8m0_value(unsigned code);
 unsigned ref_e2m1_encode(float v);
 unsigned ref_e4m3_encode(float v);
+void ref_window_fp8(const float* x, int n, uint8_t* codes);
 int ref_mx_shared_exp(float amax);
 float ref_spec_exp(float x);
 

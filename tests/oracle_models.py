@@ -39,13 +39,15 @@ def ref_model(wl, T=None):
     t = wl.table
     m = oracle.RefModel(t, wl.B, [wl.capacity_entries(s) for s in range(t.n_sources)],
                         [W.w_idx(wl, s) for s in range(t.n_sources)], wl.H, wl.H_idx, wl.K, wl.scale,
-                        pool_blocks=wl.pool_blocks)
+                        pool_blocks=wl.pool_blocks, win_fp8=wl.win_fp8)
     for s in range(t.n_sources):
         m.caches[s] = ref_cache(wl, s, range(wl.B), T)
     for l in range(t.n_layers):
         for b in range(wl.B):
             ring, cnt = ref_window(wl, l, b, T)
             m.win[l, b] = ring
+            if wl.win_fp8:
+                m.win8[l, b] = oracle.window_fp8(ring)
             m.win_count[l, b] = cnt
     return m
 
