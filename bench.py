@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=5)
+    ap.add_argument("--measure", choices=["step", "cache_io"], default="step",
+                    help="cache_io: prefix-cache export/import throughput of one source's sequences")
     return ap.parse_args()
 
 
@@ -320,14 +322,13 @@ def run_reference(args, rank):
 def run_ours(args, rank, world, local_rank):
     import ctypes
     import torch
-    import torch.distributed as dist
     import fp4_sparse_attention_pack_b200 as csa
-    from fp4_sparse_attention_pack_b200 import engine, workloads as W
+    from fp4_sparse_attention_pack_b200 import engine, replicas, workloads as W
 
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
     base = W.PROFILE_WORKLOADS[args.workload] if args.workload else W.WORKLOADS[args.config]
-    wl = W.small(base, seed=base.seed + 1000 * rank)  # each rank: its own batch of sequences
+    wl = replicas.rank_workload(base, rank)  # each rank: its own batch of sequences
     extra = args.warmup + args.steps + 2 * args.profile_steps + 8
     dm = engine.DecodeModel(wl, dev, steps_capacity=extra)
     dm.fill()
@@ -335,8 +336,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(world)
 
     stream = torch.cuda.Stream()
     torch.cuda.current_stream().wait_stream(torch.cuda.default_stream())
@@ -370,11 +370,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     time.sleep(0.25)
     clocks.stop()
-    ms = ev0.elapsed_time(ev1) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = replicas.max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
     n_ent = [dm.caches[s].n_entries.cpu().tolist() for s in range(dm.S)]
     status = dm.status_bits()
 
@@ -453,17 +449,13 @@ def run_ours(args, rank, world, local_rank):
     stream.wait_stream(s_out)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / e2e_steps if e2e_steps else float("nan")
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = replicas.max_over_ranks(f0.elapsed_time(f1) / e2e_steps if e2e_steps else float("nan"), world, dev)
     barrier()
     if rank != 0:
         return
 
     L = wl.table.n_layers
-    value = L * world / (ms / 1e3)
+    value = replicas.job_rate(L, world, ms / 1e3)
     kb = kernel_bytes(wl, n_ent)
     peak, peak_kind = measured_peaks()
     # roofline of the kernel with the largest share of the step
@@ -492,7 +484,7 @@ def run_ours(args, rank, world, local_rank):
         "kernels": kernels,
         "phase_ms": phase_ms,
         **({"phase_note": phase_note} if wl.pool_blocks > 0 else {}),
-        "e2e": {"value": L * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": replicas.job_rate(L, world, e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "method": "csa2_layer_step with every step's inputs copied from pinned host memory and "
                           "its outputs read back; two buffer sets, copies on their own streams overlap "
@@ -507,8 +499,64 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_cache_io(args):
+    """Prefix-cache export / import (csa2_cache_export / csa2_cache_import) of
+    every sequence of one source at the workload's context, into device images
+    and into pinned host images, and back into a cache with another page
+    permutation.  Prints one JSON line (GB/s of image bytes moved)."""
+    import torch
+    import fp4_sparse_attention_pack_b200 as csa
+    from fp4_sparse_attention_pack_b200 import engine, workloads as W
+    wl = W.WORKLOADS[args.config]
+    dm = engine.DecodeModel(wl, "cuda")
+    dm.fill()
+    src = dm.caches[0]
+    B, cap = wl.B, src.max_pages * 64
+    nbytes = csa.seq_image_bytes(cap)
+    dst = engine.DeviceCache(B, src.max_pages, src.ratio, "cuda", page_seed=99)
+    dev_img = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(B)]
+    host_img = [torch.empty(nbytes, dtype=torch.uint8).pin_memory() for _ in range(B)]
+    torch.cuda.synchronize()
+
+    def timed(fn, reps):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    used = sum(356 * n for n in src.n_entries.cpu().tolist())  # bytes of the sequences' entries
+    res = {}
+    for name, imgs, reps in (("device", dev_img, 20), ("pinned_host", host_img, 5)):
+        t_exp = timed(lambda: [csa.cache_export(src.desc, b, imgs[b], cap) for b in range(B)], reps)
+        t_imp = timed(lambda: [csa.cache_import(dst.desc, b, imgs[b], cap) for b in range(B)], reps)
+        res[name] = {"export_gbs": used / t_exp / 1e9, "import_gbs": used / t_imp / 1e9,
+                     "export_ms": t_exp * 1e3, "import_ms": t_imp * 1e3}
+    import numpy as np
+    ok = all(np.array_equal(a, b) for a, b in zip(dst.logical(0, 0, 1024), src.logical(0, 0, 1024)))
+    peak, peak_kind = measured_peaks()
+    ach = 2 * used / (res["device"]["export_ms"] / 1e3) / 1e9  # entries read + image written
+    line = {"metric": "prefix-cache image throughput", "unit": "GB/s", "value": res["device"]["export_gbs"],
+            "higher_is_better": True, "n_gpus": 1, "data": "synthetic",
+            "config": {"workload": wl.name, "source": 0, "sequences": B, "entries_per_sequence": wl.entries(0),
+                       "entry_bytes": 356, "image_bytes_per_sequence": nbytes},
+            "results": res, "status": src.status_bits() | dst.status_bits(),
+            "round_trip_first_1024_entries_equal": ok,
+            "roofline": {"kernel": "k_export", "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                         "frac": ach / peak, "peak_source": peak_kind, "traffic": None}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.measure == "cache_io":
+        run_cache_io(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
