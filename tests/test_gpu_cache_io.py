@@ -9,6 +9,8 @@ torch = pytest.importorskip("torch")
 
 from fp4_sparse_attention_pack_b200 import workloads as W
 
+from .oracle_models import ref_cache
+
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
@@ -74,6 +76,13 @@ def test_export_import_round_trip(csa, T):
     assert np.array_equal(img[16:16 + PEND].cpu().numpy().view(np.float32), c_src.pend_x[1].cpu().numpy())
     for got, want in zip(image_rows(img, cap, n), c_src.logical(1, 0, n)):
         assert np.array_equal(got, want)
+    # ... which are the oracle's packed entries of that sequence (same seeded recipe)
+    rc = ref_cache(wl, 0, [1], T, cap=n + 64)
+    for got, want in zip(image_rows(img, cap, n), (rc.mc[0, :n], rc.ms[0, :n], rc.kc[0, :n], rc.ks[0, :n])):
+        assert np.array_equal(got, want)
+    assert rc.pend_valid[0] == pend_valid
+    if pend_valid:
+        assert np.array_equal(img[16:16 + PEND].cpu().numpy().view(np.float32), rc.pend_x[0])
     # into sequence 0 of a cache with another page permutation
     dst = csa.engine.DeviceCache(3, c_src.max_pages, 2, DEV, page_seed=77, spare_pages=5)
     csa.cache_import(dst.desc, 0, img, cap)
