@@ -164,7 +164,7 @@ __device__ void emit_topk(KeyAt key_at, IdxAt idx_at, OutOf out_of, int cnt, uin
     }
 }
 
-__global__ void __launch_bounds__(kThreads) k_topk(const __grid_constant__ ScanBatch sb) {
+__global__ void __launch_bounds__(kThreads, 4) k_topk(const __grid_constant__ ScanBatch sb) {
     extern __shared__ uint8_t smem_raw[];
     TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
     const ScanProblem& P = sb.p[blockIdx.y];
