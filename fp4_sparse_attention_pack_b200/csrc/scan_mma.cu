@@ -257,15 +257,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // below it.n are valid, so their blocks lie below n_entries)
                 const ScanProblem& P0 = sb.p[S.prob[0]];
                 const int slots = (it.n + kPoolBlock - 1) / kPoolBlock;
+                const int n_slot = 16 * (it.t1 - it.t0);  // <= 32 * kSlotsPerLane
+                constexpr int kSlotsPerLane = kMaxChunk * 16 / 32;
                 __syncwarp();  // the previous item's reads of prow are done
-                for (int i = lane; i < 16 * (it.t1 - it.t0); i += 32) {
-                    const int slot = 16 * it.t0 + i;
+                // all of a lane's block ids, then all their page ids: two rounds of
+                // independent loads instead of a chain of dependent pairs
+                int blk[kSlotsPerLane], pg[kSlotsPerLane];
+#pragma unroll
+                for (int j = 0; j < kSlotsPerLane; ++j) {
+                    const int i = lane + 32 * j, slot = 16 * it.t0 + i;
+                    blk[j] = (i < n_slot && slot < slots) ? P0.pool[(int64_t)it.b * P0.pool_blocks + slot] : -1;
+                    if (blk[j] >= c.max_pages * (PAGE / kPoolBlock)) blk[j] = -1;  // never past the table
+                }
+#pragma unroll
+                for (int j = 0; j < kSlotsPerLane; ++j)
+                    pg[j] = blk[j] >= 0 ? c.page_table[(int64_t)it.b * c.max_pages + kPoolBlock * blk[j] / PAGE] : -1;
+#pragma unroll
+                for (int j = 0; j < kSlotsPerLane; ++j) {
+                    const int i = lane + 32 * j;
+                    if (i >= n_slot) continue;
                     int r = -1;
-                    if (slot < slots) {
-                        const int e0 = kPoolBlock * P0.pool[(int64_t)it.b * P0.pool_blocks + slot];
-                        const int pp = c.page_table[(int64_t)it.b * c.max_pages + e0 / PAGE];
-                        if (pp >= 0 && pp < c.num_pages)
-                            r = pp * PAGE + e0 % PAGE;
+                    if (blk[j] >= 0) {
+                        if (pg[j] >= 0 && pg[j] < c.num_pages)
+                            r = pg[j] * PAGE + kPoolBlock * blk[j] % PAGE;
                         else
                             atomicOr(c.status, CSA2_DEVERR_PAGE);
                     }
