@@ -208,7 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         // Lanes fetch the item's page ids (2 per tile, up to 32) in one round;
-        // one elected lane of the converged warp issues every copy.
+        // barrier arms come from one elected lane, and the copies of a tile or an
+        // item are issued by several lanes at once.
         const uint64_t pol_stream = policy_evict_first();
         const uint64_t pol_keep = policy_evict_last();
         if (lane == 0) prefetch_tmap(&mp.queries);
