@@ -75,7 +75,8 @@ constexpr int kGroups = 2;        // epilogue groups
 constexpr int kAcc = 3;           // TMEM accumulators: pass p lands in p % kAcc, group p % kGroups drains it
 constexpr int kEpiWarps = 8 * kGroups;
 constexpr int kSfWarp = 2 + kEpiWarps;
-constexpr int kThreads = 32 * (kSfWarp + 1);
+constexpr int kProducer1Warp = kSfWarp + 1;  // second producer: the odd tiles
+constexpr int kThreads = 32 * (kProducer1Warp + 1);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = 0;                            // kAcc x 128 accumulator columns
 constexpr uint32_t kColSfa = 128 * kAcc;                   // kStages x 4 scale columns (keys)
@@ -112,7 +113,7 @@ struct __align__(1024) Smem {
     uint8_t sfb_tc[2][kMaxPasses][512];
     float w[2][kMaxSub][kHeads];
     float* rows[2][kMaxSub];                 // score row of the item's sequence, per problem
-    int prow[kMaxChunk * 16];                // pool items: first physical key row of each slot
+    int prow[2][kMaxChunk * 16];             // pool items, per producer: first physical key row of each slot
     uint64_t full[kStages], empty[kStages], sfa_ready[kStages];
     uint64_t bfull[2], bempty[2], sfb_ready[2];
     uint64_t tfull[kAcc], tempty[kAcc];
@@ -205,15 +206,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        // Lanes fetch the item's page ids (2 per tile, up to 32) in one round;
-        // barrier arms come from one elected lane, and the copies of a tile or an
-        // item are issued by several lanes at once.
+    if (warp == 0 || warp == kProducer1Warp) {
+        // ------------------------------------------------------------ producers
+        // Two warps walk the same items; the CTA's tiles are numbered in order (g)
+        // and producer pw loads the tiles with g % 2 == pw into stage g % kStages
+        // (kStages is even, so every use of a stage belongs to one producer).
+        // Producer 0 also loads each item's queries.  Lanes fetch the item's page
+        // ids (2 per tile, up to 32) in one round; barrier arms come from one
+        // elected lane, and the copies of a tile or an item are issued by several
+        // lanes at once.
+        const uint32_t pw = warp == 0 ? 0u : 1u;
         const uint64_t pol_stream = policy_evict_first();
         const uint64_t pol_keep = policy_evict_last();
-        if (lane == 0) prefetch_tmap(&mp.queries);
-        uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0;
+        if (lane == 0 && pw == 0) prefetch_tmap(&mp.queries);
+        uint32_t g = 0, bslot = 0, bphase = 0;
         uint32_t issued = 0, issued_par = 0;  // per stage: a copy was issued, and its phase
         for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
             Item it;
@@ -231,7 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     atomicOr(c.status, CSA2_DEVERR_PAGE);
             }
             bool stop = false;
-            if (!mbar_wait_warp(&sm.bempty[bslot], bphase ^ 1)) {
+            if (pw != 0) {
+                // queries are producer 0's
+            } else if (!mbar_wait_warp(&sm.bempty[bslot], bphase ^ 1)) {
                 if (lane == 0) raise_abort(sm, c.status);
                 stop = true;
             } else {
@@ -284,14 +292,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         else
                             atomicOr(c.status, CSA2_DEVERR_PAGE);
                     }
-                    sm.prow[i] = r;
+                    sm.prow[pw][i] = r;
                 }
                 __syncwarp();
             }
-            for (int t = it.t0; t < it.t1 && !stop; ++t) {
+            for (int t = it.t0; t < it.t1 && !stop; ++t, ++g) {
+                if ((g & 1u) != pw) continue;
+                const uint32_t stage = g % kStages, sphase = (g / kStages) & 1u;
                 const int pg0 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0));
                 const int pg1 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0) + 1);
-                const int prow = S.pool && lane < 16 ? sm.prow[16 * (t - it.t0) + lane] : -1;
+                const int prow = S.pool && lane < 16 ? sm.prow[pw][16 * (t - it.t0) + lane] : -1;
                 const unsigned have = __ballot_sync(0xffffffffu, prow >= 0);
                 if (!mbar_wait_warp(&sm.empty[stage], sphase ^ 1)) {
                     if (lane == 0) raise_abort(sm, c.status);
@@ -313,7 +323,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     issued |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (sphase << stage);
-                    if (++stage == kStages) stage = 0, sphase ^= 1;
                     continue;
                 }
                 const uint32_t bytes = (pg0 >= 0 ? PAGE * (ICB + ISB) : 0) + (pg1 >= 0 ? PAGE * (ICB + ISB) : 0);
@@ -336,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 issued |= 1u << stage;
                 issued_par = (issued_par & ~(1u << stage)) | (sphase << stage);
-                if (++stage == kStages) stage = 0, sphase ^= 1;
             }
             if (stop) break;
         }
