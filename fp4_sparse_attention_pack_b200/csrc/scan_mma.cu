@@ -15,15 +15,16 @@
 // (two MMAs of K = 64 each).  The epilogue applies ReLU, the head weights and
 // the head sum, one thread per (entry row, problem).
 //
-// Persistent, warp-specialised CTA (608 threads, one CTA per SM):
-//   warp 0  producer: TMA tile loads of the keys (one 64-entry page per box,
-//           64-byte swizzle) and bulk copies of their E8M0 scales into an
-//           8-stage ring; per work item the query tiles, scales and head
-//           weights of every problem of the subset (double-buffered).  Keys
-//           stream with an L2 evict-first policy.  Copies are issued by several
-//           lanes at once (a lane per page, per problem or per pool block):
-//           issuing them one by one from a single lane made this warp the
-//           bottleneck of the whole pipeline.
+// Persistent, warp-specialised CTA (640 threads, one CTA per SM):
+//   warps 0, 19  producers: TMA tile loads of the keys (one 64-entry page per
+//           box, 64-byte swizzle) and bulk copies of their E8M0 scales into an
+//           8-stage ring, the two warps taking alternate tiles; warp 0 also
+//           loads per work item the query tiles, scales and head weights of
+//           every problem of the subset (double-buffered).  Keys stream with an
+//           L2 evict-first policy.  Copies are issued by several lanes at once
+//           (a lane per page, per problem or per pool block): issued one by one
+//           from a single lane of a single warp, they set the pace of the whole
+//           pipeline when a subset holds one problem.
 //   warp 1  MMA issuer: per tile issues one MMA pass per
 //           problem pair into one of three TMEM accumulators (pass p into
 //           p % 3), committing each pass to its epilogue group.  Its only
