@@ -153,3 +153,33 @@ def test_model_pool_blocks_range(capi):
         sizes[pb] = capi.layer_step_workspace(m)
     assert sizes[-1] == 0 and sizes[capi.MAX_POOL_BLOCKS + 1] == 0
     assert sizes[16] > sizes[0] > 0
+
+
+def test_layer_step_launch_counts(capi):
+    """Host-side launch accounting (no launch happens): window append, cache write (2),
+    indexer (3), attention (1 when there are at least as many (layer, sequence) units as
+    SMs -- here 1 sequence, so the split path with a combine: 2); pools add the block
+    maxima (1) and, with Reindex layers, the pool scans (4)."""
+    from fp4_sparse_attention_pack_b200 import workloads as W
+    lib = capi.lib()
+
+    def count(table, pool_blocks, with_token=True):
+        L, S = table.n_layers, table.n_sources
+        caches = (capi.csa2_cache * S)(*[capi.csa2_cache(*([16] * 10), 1, 1, 1, r) for r in table.ratios])
+        wins = (capi.csa2_window * L)(*[capi.csa2_window(16, 16, 1) for _ in range(L)])
+        ws = (ctypes.c_void_p * S)(*([16] * S))
+        keep = [(ctypes.c_int32 * L)(*table.mode), (ctypes.c_int32 * L)(*[max(s, 0) for s in table.src]),
+                (ctypes.c_int32 * L)(*[max(s, 0) for s in table.idx_src])]
+        m = capi.csa2_model(L, S, keep[0], keep[1], keep[2], caches, ws, wins, 1, 64, 64, 512, 0.04, pool_blocks)
+        x = (ctypes.c_void_p * S)(*([16 if with_token else None] * S))
+        sin = capi.csa2_step_in(x, x)
+        return lib.csa2_layer_step_launches(ctypes.byref(m), ctypes.byref(sin))
+
+    alt, pages, one = W.schedule_alternating_40(), W.schedule_pages_40(), W.single_full()
+    base = 1 + 2 + 3 + 2
+    assert count(alt, 0) == base
+    assert count(alt, 0, with_token=False) == base - 2
+    assert count(alt, 2048) == base + 1 + 4
+    assert count(pages, 2048) == base + 1 + 4
+    assert count(one, 2048) == base + 1            # a pool is built, no Reindex layer scans it
+    assert count(alt, -1) < 0                      # invalid table: a negative status
