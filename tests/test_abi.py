@@ -19,7 +19,8 @@ def capi():
 
 
 def declared_functions():
-    src = open(os.path.join(ROOT, "include", "csa2.h")).read()
+    with open(os.path.join(ROOT, "include", "csa2.h")) as f:
+        src = f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(csa2_[a-z0-9_]+)\s*\(", src)))
 

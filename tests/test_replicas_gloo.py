@@ -40,7 +40,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_shard_by_sequence_and_time_by_the_slowest():
     world = 2
-    with mp.Manager() as man:
+    with mp.get_context("spawn").Manager() as man:
         out = man.dict()
         mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
         res = dict(out)
