@@ -247,7 +247,8 @@ int csa2_index_topk_pool(const csa2_cache* cache, const uint16_t* q_idx, const f
  * block ids, then -1); block ids that are negative or at or beyond the
  * sequence's blocks end the pool early.  A pool in another order gives a
  * selection among its blocks' entries whose order and tie rule are not
- * specified.  Same workspace and errors as csa2_index_topk_pool.
+ * specified, and a block listed twice can give an index twice.  Same
+ * workspace and errors as csa2_index_topk_pool (INVALID_ARG for a NULL pool).
  */
 int csa2_index_topk_in_pool(const csa2_cache* cache, const uint16_t* q_idx, const float* w,
                             int H_idx, int K, const int32_t* pool, int pool_blocks,
