@@ -208,10 +208,11 @@ WIN = 128
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_sample(wl, seqs=(0,), layers=None, budget_s=None):
+def oracle_sample(wl, seqs=(0,), layers=None, scores_out=None):
     """Time the oracle on `layers` for `seqs` (caches built untimed).  Returns
     (seconds per (scan layer, sequence), seconds per (attention-only layer,
-    sequence), threads, description)."""
+    sequence), threads, description).  scores_out (a dict, optional) receives the
+    oracle's fp64 indexer scores of every scan layer of the first sequence."""
     import numpy as np
     import oracle
     from fp4_sparse_attention_pack_b200 import workloads as W
@@ -231,6 +232,8 @@ def oracle_sample(wl, seqs=(0,), layers=None, budget_s=None):
                 c = caches[t.src[l]]
                 sc = c.scores(i, W.query_idx(wl, l, 0)[b], W.head_weights(wl, l, 0)[b])
                 idx[l] = oracle.topk(sc, wl.K)
+                if scores_out is not None and i == 0:
+                    scores_out[l] = sc
             sel = idx.get(l if m != W.REUSE else t.idx_src[l])
             if m == W.SWA_ONLY:
                 items = oracle.attention_items(np.zeros((1, 256), np.uint8), np.zeros((1, 32), np.uint8),
@@ -250,13 +253,34 @@ def oracle_sample(wl, seqs=(0,), layers=None, budget_s=None):
             oracle.threads(), desc)
 
 
-def cpu_baseline(wl):
-    ts, ta, thr, desc = oracle_sample(wl)
+def cpu_baseline(wl, gpu_first_idx=None):
+    """The oracle's sampled rate; with gpu_first_idx ([layers][K] indices of the
+    GPU's first step for sequence 0), also the Top-K parity of those layers
+    against the oracle's scores, with the tie-band counts."""
+    scores = {}
+    ts, ta, thr, desc = oracle_sample(wl, scores_out=scores)
     n_scan = len(wl.table.scan_layers())
     n_attn = wl.table.n_layers - n_scan
     step_s = wl.B * (n_scan * ts + n_attn * ta)
-    return {"value": wl.table.n_layers / step_s, "unit": UNIT, "cores": thr, "kind": "oracle",
+    base = {"value": wl.table.n_layers / step_s, "unit": UNIT, "cores": thr, "kind": "oracle",
             "sample": desc}
+    parity = None
+    if gpu_first_idx is not None and scores:
+        from tests.parity import TOPK_REL, topk_tie_report
+        band = differ = 0
+        ok = True
+        for l, sc in sorted(scores.items()):
+            try:
+                r = topk_tie_report(gpu_first_idx[l], sc, wl.K)
+                band += r["band"]
+                differ += r["differ"]
+            except AssertionError:
+                ok = False
+        parity = {"topk_rows_checked": len(scores), "topk_sets_match": ok, "tie_band_rel": TOPK_REL,
+                  "tie_band_entries": band, "indices_differ": differ,
+                  "rows": f"sequence 0 of layers {sorted(scores)} at the first decode step, GPU indices "
+                          f"against the oracle's fp64 scores"}
+    return base, parity
 
 
 # ---------------------------------------------------------------- reference arm
@@ -344,6 +368,7 @@ def run_ours(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         dm.step(stream)
     stream.synchronize()
+    first_idx = dm.idx[:, 0].cpu().numpy() if world == 1 else None  # the oracle sample's step
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         dm.step(torch.cuda.current_stream())
@@ -495,7 +520,10 @@ def run_ours(args, rank, world, local_rank):
         "device_status": status,
     }
     if world == 1 and not args.no_cpu_baseline and not args.workload:
-        line["cpu_baseline"] = cpu_baseline(W.WORKLOADS[args.config])
+        line["cpu_baseline"], parity = cpu_baseline(W.WORKLOADS[args.config],
+                                                    first_idx if wl.pool_blocks == 0 else None)
+        if parity is not None:
+            line["parity"] = parity
     print(json.dumps(line), flush=True)
 
 

@@ -6,6 +6,8 @@
 // Everything is validated before the first launch, so an error return means
 // nothing was enqueued.  Nothing is allocated and nothing synchronises, so
 // every entry point can be captured in a CUDA graph.
+#include <atomic>
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -14,12 +16,33 @@
 using namespace csa2;
 
 namespace {
+std::atomic<int> g_injected_faults{0};
+}  // namespace
+
+bool csa2::inject_fault(const char* entry) {
+    const char* v = std::getenv("CSA2_INJECT_FAULT");
+    if (!v || !*v) return false;
+    const size_t n = std::strlen(entry);
+    bool hit = false;
+    for (const char* p = v; *p && !hit;) {
+        const char* e = std::strchr(p, ',');
+        const size_t len = e ? (size_t)(e - p) : std::strlen(p);
+        hit = (len == 1 && p[0] == '*') || (len == n && std::strncmp(p, entry, n) == 0);
+        p = e ? e + 1 : p + len;
+    }
+    if (hit) g_injected_faults.fetch_add(1, std::memory_order_relaxed);
+    return hit;
+}
+
+namespace {
 
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_cache(const csa2_cache* c) {
+}  // namespace
+
+int csa2::check_cache(const csa2_cache* c) {
     if (!c) return CSA2_ERR_INVALID_ARG;
     if (!c->main_codes || !c->main_scales || !c->idx_codes || !c->idx_scales || !c->page_table ||
         !c->n_entries || !c->pend_x || !c->pend_g || !c->pend_valid || !c->status)
@@ -33,6 +56,8 @@ int check_cache(const csa2_cache* c) {
         return CSA2_ERR_ALIGN;
     return CSA2_OK;
 }
+
+namespace {
 
 int check_window(const csa2_window* w, int batch) {
     if (!w || !w->tokens || !w->count || w->batch != batch) return CSA2_ERR_INVALID_ARG;
@@ -52,6 +77,8 @@ size_t topk_ws_one(int batch, int max_entries, int H_idx) {
 extern "C" {
 
 int csa2_version(void) { return (0 << 16) | 1; }
+
+int csa2_injected_faults(void) { return g_injected_faults.load(std::memory_order_relaxed); }
 
 const char* csa2_strerror(int status) {
     switch (status) {
@@ -83,6 +110,7 @@ int csa2_pack_cache(const csa2_cache* cache, const void* x, int x_dtype, const f
     pb.x[0] = x;
     pb.gates[0] = gates;
     pb.W[0] = w_idx;
+    if (inject_fault("csa2_pack_cache")) return CSA2_ERR_CUDA;
     return cuda_status(launch_pack(pb, x_dtype == CSA2_DTYPE_F32, T_new, (cudaStream_t)stream));
 }
 
@@ -116,6 +144,7 @@ int csa2_index_topk(const csa2_cache* cache, const uint16_t* q_idx, const float*
     P.idx_out = idx_out;
     P.score_out = score_out;
     carve_scan_workspace(sb, static_cast<uint8_t*>(ws), cache->batch, cap);
+    if (inject_fault("csa2_index_topk")) return CSA2_ERR_CUDA;
     return cuda_status(launch_index_topk(sb, (cudaStream_t)stream));
 }
 
@@ -186,6 +215,7 @@ int csa2_index_topk_pool(const csa2_cache* cache, const uint16_t* q_idx, const f
     sb.p[0].idx_out = idx_out;
     sb.p[0].score_out = score_out;
     carve_scan_workspace(sb, wsp, cache->batch, pw.rows);
+    if (inject_fault("csa2_index_topk_pool")) return CSA2_ERR_CUDA;
     rc = cuda_status(launch_quant_scan(sb, st));
     if (rc) return rc;
     float* bmax = reinterpret_cast<float*>(wsp + pw.scan);
@@ -227,6 +257,7 @@ int csa2_index_topk_in_pool(const csa2_cache* cache, const uint16_t* q_idx, cons
     P.pool_blocks = pool_blocks;
     P.pool_n = reinterpret_cast<int32_t*>(wsp + pw.scan + pw.bmax);
     carve_scan_workspace(sb, wsp, cache->batch, pw.rows);
+    if (inject_fault("csa2_index_topk_in_pool")) return CSA2_ERR_CUDA;
     return cuda_status(launch_index_topk(sb, (cudaStream_t)stream));
 }
 
@@ -273,6 +304,7 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const in
     P.win_count = win->count;
     P.out = out;
     P.K = K;
+    if (inject_fault("csa2_sparse_attn")) return CSA2_ERR_CUDA;
     return cuda_status(launch_sparse_attn(ab, (cudaStream_t)stream));
 }
 
@@ -290,6 +322,7 @@ int csa2_window_append(const csa2_window* win, const uint16_t* tok, csa2_stream 
     wa.fp8[0] = win->dtype == CSA2_WIN_FP8;
     wa.count[0] = win->count;
     wa.tok[0] = tok;
+    if (inject_fault("csa2_window_append")) return CSA2_ERR_CUDA;
     return cuda_status(launch_window_append(wa, (cudaStream_t)stream));
 }
 
@@ -438,6 +471,7 @@ int layer_step_impl(const csa2_model* m, const csa2_step_in* in, const csa2_step
     const size_t need = csa2_layer_step_workspace(m);
     if (!ws || ws_bytes < need) return CSA2_ERR_WORKSPACE;
     if (!a16(ws)) return CSA2_ERR_ALIGN;
+    if (inject_fault(ev ? "csa2_layer_step_profiled" : "csa2_layer_step")) return CSA2_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     if (ev) cudaEventRecord(ev[0], st);
 

@@ -1,6 +1,6 @@
-// Sparse + window attention ("la requête (main Q) lit les entrées
-// sélectionnées et le KV SWA local de la couche"; main KV "décompressé avant
-// l'attention"), the SWA ring write, and the split combine.
+// Sparse + window attention (CSA2 chapter of "DeepSeek-V4.1-Flash, expliqué pas
+// à pas": the main query reads the selected entries, decompressed, and the
+// layer's local SWA KV), the SWA ring write, and the split combine.
 //
 // Items of (problem, sequence): positions [0, K) are the selected entries
 // (index -1 or beyond n_entries is masked), positions [K, K + 128) the window
@@ -231,11 +231,9 @@ namespace {
 // CUDA-core path (heads beyond the tensor-core kernel's 64).
 cudaError_t launch_attn_cuda(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev) {
     const size_t smem = sizeof(float) * (kSplit * kStride + kWarps * D);
-    static const bool attr_set = [smem] {
-        cudaFuncSetAttribute(k_attn_split, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        return true;
-    }();
-    (void)attr_set;
+    static std::atomic<uint64_t> attr_done{0};
+    const cudaError_t ea = smem_opt_in(reinterpret_cast<const void*>(k_attn_split), (int)smem, attr_done);
+    if (ea != cudaSuccess) return ea;
     dim3 grid(n_splits(ab.Kmax), ab.batch, ab.n);
     k_attn_split<<<grid, kThreads, smem, st>>>(ab);
     cudaError_t e = cudaGetLastError();

@@ -214,7 +214,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tbase = sm.tmem_base;
+    // lane 0's copy: a value the compiler knows is warp-uniform, so the MMA
+    // operands derived from it need no per-lane handling at issue
+    const uint32_t tbase = __shfl_sync(0xffffffffu, sm.tmem_base, 0);
     uint32_t phase = 0, wphase = 0;
     bool o_init = false;
     bool timed_out = false;
@@ -568,16 +570,6 @@ __global__ void k_attn_mma_combine(const __grid_constant__ AttnBatch ab, int spl
     for (int i = 0; i < 4; ++i) o[threadIdx.x + 128 * i] = acc[i] * inv;
 }
 
-int sm_count_attn() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
 
 }  // namespace
 
@@ -586,7 +578,7 @@ int sm_count_attn() {
 int attn_mma_splits(int n_problems, int batch, int Kmax) {
     const int tiles = (Kmax + WIN + kT - 1) / kT;
     const int pairs = n_problems * batch;
-    const int want = (sm_count_attn() + pairs - 1) / pairs;
+    const int want = (device_sm_count() + pairs - 1) / pairs;
     return std::max(1, std::min(tiles, want));
 }
 
@@ -642,11 +634,9 @@ cudaError_t launch_attn_mma(const AttnBatch& ab_in, cudaStream_t st, cudaEvent_t
         ab.part_ml = ab.part_o + units * ab.H * D;
     }
     const size_t smem = sizeof(Smem) + 1024;
-    static const bool attr = [smem] {
-        cudaFuncSetAttribute(k_attn_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        return true;
-    }();
-    (void)attr;
+    static std::atomic<uint64_t> attr_done{0};
+    const cudaError_t ea = smem_opt_in(reinterpret_cast<const void*>(k_attn_mma), (int)smem, attr_done);
+    if (ea != cudaSuccess) return ea;
     k_attn_mma<<<ab.n * ab.batch * splits, kThreads, smem, st>>>(ab, maps, splits, tps);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -160,6 +160,7 @@ extern "C" size_t csa2_seq_image_bytes(int capacity) {
 extern "C" int csa2_cache_export(const csa2_cache* cache, int seq, void* image, int capacity, csa2_stream stream) {
     const int rc = csa2::check_io(cache, seq, image, capacity);
     if (rc) return rc;
+    if (csa2::inject_fault("csa2_cache_export")) return CSA2_ERR_CUDA;
     return csa2::launch_io(cache, seq, image, capacity, stream, true);
 }
 
@@ -167,5 +168,6 @@ extern "C" int csa2_cache_import(const csa2_cache* cache, int seq, const void* i
                                  csa2_stream stream) {
     const int rc = csa2::check_io(cache, seq, image, capacity);
     if (rc) return rc;
+    if (csa2::inject_fault("csa2_cache_import")) return CSA2_ERR_CUDA;
     return csa2::launch_io(cache, seq, const_cast<void*>(image), capacity, stream, false);
 }

@@ -1,9 +1,46 @@
 // Internal launchers of the CSA2 kernels (host side of csrc/*.cu).
 #pragma once
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace csa2 {
+
+// Opt `func` into `bytes` of dynamic shared memory on the current device.  The
+// attribute is per device, so it is set once per device (bit d of `done`) and
+// its error is returned; devices 64 and up set it on every call.
+inline cudaError_t smem_opt_in(const void* func, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
+// Host-side checks of a cache descriptor made before any launch: CSA2_OK, or
+// CSA2_ERR_INVALID_ARG (a null pointer, a bad size or ratio), CSA2_ERR_ALIGN (a
+// pointer not 16-byte aligned) or CSA2_ERR_UNSUPPORTED (capacity beyond 2^30).
+int check_cache(const csa2_cache* c);
+
+// Host-side fault injection for tests of callers' error paths: true when the
+// environment variable CSA2_INJECT_FAULT names `entry` (a comma-separated list
+// of entry-point names, or "*" for all).  The entry point then returns
+// CSA2_ERR_CUDA after its argument checks and before its first launch, as if
+// the launch had failed.  Unset (the default), it costs one getenv per call.
+bool inject_fault(const char* entry);
+
+// Multiprocessors of the current device (148 when the query fails).
+inline int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    return n;
+}
 
 // ---- cache write: the same T new tokens per sequence for each listed source
 constexpr int kMaxPackSources = 8;

@@ -58,22 +58,16 @@ extern "C" int csa2_index_topk_noalloc(const csa2_cache* cache, const uint16_t* 
                                        int H_idx, int K, int32_t* idx_out, float* score_out,
                                        csa2_stream stream) {
     using namespace csa2;
-    if (!cache || !q_idx || !w || !idx_out) return CSA2_ERR_INVALID_ARG;
-    if (!cache->main_codes || !cache->main_scales || !cache->idx_codes || !cache->idx_scales ||
-        !cache->page_table || !cache->n_entries || !cache->pend_x || !cache->pend_g ||
-        !cache->pend_valid || !cache->status)
-        return CSA2_ERR_INVALID_ARG;
-    if (cache->batch < 1 || cache->max_pages < 1 || cache->num_pages < 1 ||
-        (cache->ratio != 1 && cache->ratio != 2))
-        return CSA2_ERR_INVALID_ARG;
+    // the same checks, in the same order, as csa2_index_topk; then the size limit
+    int rc0 = check_cache(cache);
+    if (rc0) return rc0;
     if (H_idx < 1 || H_idx > CSA2_MAX_H_IDX || K < 1 || K > CSA2_MAX_K) return CSA2_ERR_INVALID_ARG;
-    if (!aligned16(cache->idx_codes) || !aligned16(cache->idx_scales) || !aligned16(cache->page_table) ||
-        !aligned16(cache->n_entries) || !aligned16(cache->status) || !aligned16(q_idx) ||
-        !aligned16(w) || !aligned16(idx_out) || (score_out && !aligned16(score_out)))
+    if (!q_idx || !w || !idx_out) return CSA2_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(w) || !aligned16(idx_out) || (score_out && !aligned16(score_out)))
         return CSA2_ERR_ALIGN;
-    if ((int64_t)cache->max_pages * PAGE > (int64_t)1 << 30) return CSA2_ERR_UNSUPPORTED;
     const int cap = cache->max_pages * PAGE;
     if (scan_workspace_bytes(1, cache->batch, cap, H_idx) > kNoAllocBytes) return CSA2_ERR_UNSUPPORTED;
+    if (inject_fault("csa2_index_topk_noalloc")) return CSA2_ERR_CUDA;
     void* scratch = nullptr;
     const int rc = scratch_address(&scratch);
     if (rc) return rc;

@@ -244,12 +244,11 @@ cudaError_t launch_pack(const PackBatch& pb, bool x_f32, int T, cudaStream_t st)
     const int chunks = (max_new + kEnt - 1) / kEnt;
     const int batch = pb.cache[0].batch;
     const size_t smem = sizeof(float) * (kEnt * D + 2 * kWc * DI);
-    static const bool attr_set = [smem] {
-        cudaFuncSetAttribute(k_pack_entries<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        cudaFuncSetAttribute(k_pack_entries<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        return true;
-    }();
-    (void)attr_set;
+    static std::atomic<uint64_t> attr_done_f32{0}, attr_done_bf16{0};
+    const cudaError_t ea =
+        x_f32 ? smem_opt_in(reinterpret_cast<const void*>(k_pack_entries<true>), (int)smem, attr_done_f32)
+              : smem_opt_in(reinterpret_cast<const void*>(k_pack_entries<false>), (int)smem, attr_done_bf16);
+    if (ea != cudaSuccess) return ea;
     dim3 grid(chunks, batch, pb.n);
     if (x_f32)
         k_pack_entries<true><<<grid, kThreads, smem, st>>>(pb, T);

@@ -1,6 +1,7 @@
-// Indexer scan ("un indexeur léger : il note chaque entrée du main KV en
-// combinant une indexer Q et une indexer K") over MXFP4 keys and queries, and
-// the per-sequence Top-K ("puis garde les 512 meilleures").
+// Indexer scan (the pages' light indexer scores every main-KV entry from an
+// indexer query and an indexer key: "DeepSeek-V4.1-Flash, expliqué pas à pas",
+// CSA2 chapter) over MXFP4 keys and queries, and the per-sequence Top-K of the
+// 512 best entries.
 //
 //   score[b][e] = sum_h w[b][h] * max(0, qhat[b][h] . khat[b][e])
 //

@@ -142,6 +142,11 @@ __device__ __forceinline__ bool item_at(const ScanBatch& sb, const MmaScanMaps& 
     const int tiles = (it.n + kTile - 1) / kTile;
     it.t0 = c * S.chunk;
     it.t1 = min(it.t0 + S.chunk, tiles);
+    // Lane 0's values for the whole warp: the compiler then sees every loop
+    // bound and ring index derived from them as warp-uniform, so the tcgen05
+    // operands built from them need no per-lane handling at issue.
+    it.n = __shfl_sync(0xffffffffu, it.n, 0);
+    it.t1 = __shfl_sync(0xffffffffu, it.t1, 0);
     return it.t0 < it.t1;
 }
 
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tbase = sm.tmem_base;
+    const uint32_t tbase = __shfl_sync(0xffffffffu, sm.tmem_base, 0);  // warp-uniform (see item_at)
 
     if (warp == 0 || warp == kProducer1Warp) {
         // ------------------------------------------------------------ producers
@@ -546,16 +551,6 @@ bool make_rows64_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t b
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
 
 }  // namespace
 
@@ -632,7 +627,7 @@ cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st) {
     // Tiles per work item: about 64 tile-problems of work each (so subsets of
     // different sizes cost about the same per item), fewer when the items would
     // not fill the grid a few times over.
-    const int grid_max = sm_count();
+    const int grid_max = device_sm_count();
     int items = 0;
     for (int base = 64;; base /= 2) {
         items = 0;
@@ -650,11 +645,9 @@ cudaError_t launch_scan_mma(const ScanBatch& sb, cudaStream_t st) {
     mp.n_items = items;
     const int grid = std::min(items, grid_max);
     const size_t smem = sizeof(Smem) + 1024;
-    static const bool attr = [smem] {
-        cudaFuncSetAttribute(k_scan_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        return true;
-    }();
-    (void)attr;
+    static std::atomic<uint64_t> attr_done{0};
+    const cudaError_t ea = smem_opt_in(reinterpret_cast<const void*>(k_scan_mma), (int)smem, attr_done);
+    if (ea != cudaSuccess) return ea;
     k_scan_mma<<<grid, kThreads, smem, st>>>(sb, mp);
     return cudaGetLastError();
 }

@@ -1,4 +1,6 @@
-// Per-sequence Top-K of the indexer scores ("n'en garde que les 512 meilleures").
+// Per-sequence Top-K of the indexer scores (the pages' indexer keeps the 512
+// best-scoring entries: "DeepSeek-V4.1-Flash, expliqué pas à pas", attention
+// taxonomy).
 //
 // Scores map to order-preserving uint32 keys; the K largest are kept, equal
 // scores lower index first, and written in increasing index order.  A row is a
@@ -262,11 +264,9 @@ __global__ void __launch_bounds__(kThreads, 4) k_topk(const __grid_constant__ Sc
 cudaError_t launch_topk(const ScanBatch& sb, cudaStream_t st) {
     const int batch = sb.p[0].cache.batch;
     const size_t smem = sizeof(TopkSmem);
-    static const bool attr = [smem] {
-        cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        return true;
-    }();
-    (void)attr;
+    static std::atomic<uint64_t> attr_done{0};
+    const cudaError_t ea = smem_opt_in(reinterpret_cast<const void*>(k_topk), (int)smem, attr_done);
+    if (ea != cudaSuccess) return ea;
     dim3 grid(batch, sb.n);
     k_topk<<<grid, kThreads, smem, st>>>(sb);
     return cudaGetLastError();

@@ -129,9 +129,9 @@ typedef struct {
 } csa2_cache;
 
 /*
- * One layer's SWA window for `batch` sequences ("une branche locale SWA qui
- * maintient le KV SWA des 128 derniers tokens"): a ring of 128 tokens of 512
- * channels.  Token number t (0-based, counted per sequence) sits in slot
+ * One layer's SWA window for `batch` sequences (CSA2 chapter of "DeepSeek-V4.1-
+ * Flash, expliqué pas à pas": a local SWA branch keeps the KV of the last 128
+ * tokens): a ring of 128 tokens of 512 channels.  Token number t (0-based, counted per sequence) sits in slot
  * t % 128; count[b] tokens were appended, the first min(count[b], 128) slots
  * are valid.  Attention is order-free, so the ring needs no rotation.
  *
@@ -156,13 +156,26 @@ typedef struct {
 /* Library version, (major << 16) | minor. */
 int csa2_version(void);
 
+/*
+ * Host-side fault injection, for testing a caller's error paths without a GPU
+ * fault.  (The pages have no counterpart.)  When the environment variable
+ * CSA2_INJECT_FAULT holds a comma-separated list of entry-point names (or "*"
+ * for all of them), each listed entry point that launches work returns
+ * CSA2_ERR_CUDA after its argument checks and before anything is enqueued, as
+ * if its launch had failed; argument errors still take precedence.  Unset, it
+ * does nothing.  csa2_injected_faults() counts the injected failures of the
+ * process so far.
+ */
+int csa2_injected_faults(void);
+
 /* Static string for a csa2_status value (never NULL). */
 const char* csa2_strerror(int status);
 
 /*
- * Cache write ("CSA2 supprime le chevauchement" -- disjoint groups; "CSA2
- * obtient l'indexer K par une simple projection du main KV"; "Le cache KV en
- * FP4").  Appends T_new tokens to every sequence of `cache`:
+ * Cache write ("DeepSeek-V4.1-Flash, expliqué pas à pas", CSA2 chapter: token
+ * groups no longer overlap, and the indexer key is a plain projection of the
+ * main KV; chapter "Le cache KV en FP4" for the formats).  Appends T_new tokens
+ * to every sequence of `cache`:
  *   x       [batch][T_new][512] tokens, bf16 or fp32 per x_dtype (the
  *           post-RoPE latent of the source layer);
  *   gates   fp32 [batch][T_new], one gate logit per token;
@@ -187,9 +200,10 @@ int csa2_pack_cache(const csa2_cache* cache, const void* x, int x_dtype, const f
 size_t csa2_index_topk_workspace(int batch, int max_entries, int H_idx, int K);
 
 /*
- * Indexer scan + Top-K ("un indexeur léger : il note chaque entrée du main KV
- * en combinant une indexer Q et une indexer K, puis garde les 512 meilleures";
- * indexer queries and keys in OCP MXFP4).  For every sequence b:
+ * Indexer scan + Top-K (CSA2 chapter of "DeepSeek-V4.1-Flash, expliqué pas à
+ * pas": a light indexer scores every main-KV entry from an indexer query and
+ * an indexer key and keeps the best 512; indexer queries and keys in OCP
+ * MXFP4).  For every sequence b:
  *   score[e] = sum_h w[b][h] * max(0, qhat[b][h] . khat[e]),  e < n_entries[b],
  * qhat = MXFP4 of q_idx (same rule as the keys), khat the stored keys.
  * The K highest scores are kept (equal scores: lower index first); idx_out
@@ -259,9 +273,10 @@ int csa2_index_topk_in_pool(const csa2_cache* cache, const uint16_t* q_idx, cons
 size_t csa2_sparse_attn_workspace(int batch, int H, int K);
 
 /*
- * Sparse + window attention ("l'attention principale : la requête (main Q)
- * lit les entrées sélectionnées et le KV SWA local de la couche"; entries are
- * "décompressées avant l'attention").  For every sequence b and head h:
+ * Sparse + window attention ("DeepSeek-V4.1-Flash, expliqué pas à pas", CSA2
+ * chapter, main attention: the main query reads the selected entries together
+ * with the layer's local SWA KV, and the FP4 entries are decompressed before
+ * attention).  For every sequence b and head h:
  *   items = dequantised entries idx[b][0..K) (index -1 skipped; indices at or
  *           beyond n_entries[b] skipped) followed by the valid window tokens;
  *   out[b][h] = sum_j softmax_j(scale * q[b][h] . item_j) * item_j
@@ -279,8 +294,9 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const in
 int csa2_window_append(const csa2_window* win, const uint16_t* tok, csa2_stream stream);
 
 /*
- * A stack of layers and its static mode table ("Chaque couche CSA2 reçoit, de
- * façon statique, l'un des trois modes"; "Résumé exécutif" mode table):
+ * A stack of layers and its static mode table (CSA2 chapter of "DeepSeek-V4.1-
+ * Flash, expliqué pas à pas": each layer is given one of the three modes once,
+ * statically; "Résumé exécutif", mode table):
  *   mode[l]     csa2_mode of layer l;
  *   src[l]      the source cache layer l reads (ignored for SWA_ONLY);
  *   idx_src[l]  for REUSE: the earlier FULL/REINDEX layer of the same source
@@ -358,8 +374,11 @@ int csa2_layer_step(const csa2_model* model, const csa2_step_in* in, const csa2_
  *     batch * H_idx * 68 bytes, must fit in 8 MiB; larger requests return
  *     CSA2_ERR_UNSUPPORTED before anything is launched.
  *   - Set-up: the first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current).  Make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and keeps it for the
+ *     life of the process.  Make that first call before any stream capture.
+ *     The kept address belongs to the device's current context: after a
+ *     cudaDeviceReset of that device it is stale, so do not call this entry
+ *     point on a device that has been reset.
  *   - Sharing: every call uses the same array and leaves its contents behind
  *     (nothing in it needs to start at zero).  Calls whose kernels overlap on
  *     the GPU -- other streams or other host threads -- race; serialise them.

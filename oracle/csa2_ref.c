@@ -27,7 +27,8 @@ int ref_threads(void) {
 
 /* E2M1 (OCP MX v1.0, FP4): 1 sign, 2 exponent (bias 1), 1 mantissa bit.
  * Exponent 0 is subnormal: 0 or 0.5.  Eight magnitudes: 0, .5, 1, 1.5, 2, 3, 4, 6
- * ("Le cache KV en FP4": "Il ne peut représenter que 8 amplitudes"). */
+ * (the FP4 section of "DeepSeek-V4.1-Flash, expliqué pas à pas" notes that the
+ * format has only eight magnitudes). */
 double ref_e2m1_value(unsigned code) {
     unsigned s = (code >> 3) & 1u, e = (code >> 1) & 3u, m = code & 1u;
     double mag = (e == 0) ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, (int)e - 1);
@@ -132,8 +133,9 @@ float ref_spec_exp(float x) {
 
 /* -------------------------------------------------------------- cache write */
 
-/* Ratio-2 compression of one disjoint token pair (2j, 2j+1) ("CSA2 supprime le
- * chevauchement"): e = w0*x0 + w1*x1 with (w0, w1) = softmax(g0, g1), one
+/* Ratio-2 compression of one disjoint token pair (2j, 2j+1) (CSA2 chapter of
+ * "DeepSeek-V4.1-Flash, expliqué pas à pas": CSA2 drops the overlap between
+ * groups): e = w0*x0 + w1*x1 with (w0, w1) = softmax(g0, g1), one
  * scalar gate logit per token.  fp32: w0 = 1/(1 + exp(g1 - g0)), w1 = 1 - w0,
  * e_c = fma(w1, x1_c, w0*x0_c). */
 void ref_compress_pair(const float* x0, float g0, const float* x1, float g1, float* e) {
@@ -168,8 +170,9 @@ void ref_pack_main(const float* e, uint8_t* codes, uint8_t* scales) {
     }
 }
 
-/* Dequantised main entry (used before attention, "décompressées avant
- * l'attention"): E2M1 value times its E4M3 scale; exact in fp32. */
+/* Dequantised main entry (the FP4 entries are decompressed before attention:
+ * CSA2 chapter of "DeepSeek-V4.1-Flash, expliqué pas à pas"): E2M1 value times
+ * its E4M3 scale; exact in fp32. */
 void ref_dequant_main(const uint8_t* codes, const uint8_t* scales, float* out) {
     for (int c = 0; c < 512; ++c) {
         unsigned q = (codes[c >> 1] >> (4 * (c & 1))) & 15u;
@@ -204,7 +207,8 @@ void ref_mxfp4_quant(const float* v, int n, uint8_t* codes, uint8_t* scales) {
 }
 
 /* Indexer key = plain projection of the (stored, dequantised) main entry
- * ("CSA2 obtient l'indexer K par une simple projection du main KV"), then
+ * (CSA2 chapter of "DeepSeek-V4.1-Flash, expliqué pas à pas": the indexer key
+ * is a simple projection of the main KV), then
  * MXFP4.  k_o = sum_c W[c][o] * deq_c accumulated as fp32 fused multiply-adds
  * in the order c = 0, 1, ..., 511 starting from +0. */
 void ref_index_key(const uint8_t* codes, const uint8_t* scales, const float* W, uint8_t* kc,
@@ -267,8 +271,8 @@ static double mx_elem(const uint8_t* codes, const uint8_t* scales, int c) {
     return ref_e2m1_value(q) * ref_e8m0_value(scales[c >> 5]);
 }
 
-/* Indexer score of every entry ("un indexeur léger : il note chaque entrée du
- * main KV en combinant une indexer Q et une indexer K"):
+/* Indexer score of every entry (the light indexer of the CSA2 chapter scores
+ * every main-KV entry from an indexer query and an indexer key):
  * score_e = sum_h w_h * max(0, qhat_h . khat_e), query and key both MXFP4 (the
  * pages: V4 stored the indexer queries and keys in FP4).  fp64; every product
  * of two MXFP4 values is exact. */
@@ -310,7 +314,8 @@ static int cmp_i32(const void* a, const void* b) {
     return (x > y) - (x < y);
 }
 
-/* Top-K ("n'en garde que les 512 meilleures"): order all entries by score,
+/* Top-K (the indexer keeps the 512 best entries: "DeepSeek-V4.1-Flash, expliqué
+ * pas à pas", attention taxonomy): order all entries by score,
  * higher first, equal scores by lower index first; keep the first min(K, N).
  * Output: the kept indices in increasing index order, then -1 padding to K. */
 void ref_topk(const double* scores, int N, int K, int32_t* out) {
@@ -353,8 +358,8 @@ int ref_gather_items(const uint8_t* mc, const uint8_t* ms, int n_entries, const 
     return m;
 }
 
-/* Main attention over the gathered items ("la requête (main Q) lit les entrées
- * sélectionnées et le KV SWA local"): the latent item serves as both key and
+/* Main attention over the gathered items (CSA2 chapter: the main query reads
+ * the selected entries and the layer's local SWA KV): the latent item serves as both key and
  * value (MLA-style shared latent).  Plain softmax in fp64:
  * o_h = sum_j softmax_j(scale * q_h . item_j) * item_j.  M == 0 gives zeros. */
 void ref_attention(const float* q, int H, const float* items, int M, double scale, float* out) {

@@ -17,7 +17,16 @@ ATTN_REL = 2e-3
 
 
 def check_topk(gpu_idx: np.ndarray, ref_scores: np.ndarray, K: int) -> int:
-    """Assert the Top-K criterion for one sequence; return the tie-band count."""
+    """Assert the Top-K criterion for one sequence; return how many indices differ
+    from the oracle's set (each of them inside the tie band)."""
+    return topk_tie_report(gpu_idx, ref_scores, K)["differ"]
+
+
+def topk_tie_report(gpu_idx: np.ndarray, ref_scores: np.ndarray, K: int) -> dict:
+    """Assert the Top-K criterion for one sequence and report the tie band:
+    band = entries whose oracle score lies within TOPK_REL of the oracle's K-th
+    score (the entries on which the two sides may legitimately differ), differ =
+    indices in exactly one of the two sets (all of them inside the band)."""
     n = ref_scores.size
     gpu_idx = np.asarray(gpu_idx, np.int64)
     m = min(K, n)
@@ -26,7 +35,7 @@ def check_topk(gpu_idx: np.ndarray, ref_scores: np.ndarray, K: int) -> int:
     assert np.all((g >= 0) & (g < n)), "index out of range"
     assert np.all(np.diff(g) > 0), "indices must be distinct and increasing"
     if m == 0:
-        return 0
+        return {"band": 0, "differ": 0}
     order = sorted(range(n), key=lambda i: (-ref_scores[i], i)) if n < 4096 else \
         np.lexsort((np.arange(n), -ref_scores))
     ref_set = set(int(i) for i in order[:m])
@@ -35,7 +44,7 @@ def check_topk(gpu_idx: np.ndarray, ref_scores: np.ndarray, K: int) -> int:
     diff = ref_set.symmetric_difference(set(int(i) for i in g))
     bad = [i for i in diff if not band[i]]
     assert not bad, f"{len(bad)} Top-K entries differ outside the tie band, e.g. {bad[:5]}"
-    return len(diff)
+    return {"band": int(band.sum()), "differ": len(diff)}
 
 
 def attn_rel_err(out: np.ndarray, ref: np.ndarray) -> float:

@@ -184,3 +184,44 @@ def test_layer_step_launch_counts(capi):
     assert count(pages, 2048) == base + 1 + 4
     assert count(one, 2048) == base + 1            # a pool is built, no Reindex layer scans it
     assert count(alt, -1) < 0                      # invalid table: a negative status
+
+
+def test_host_fault_hook_returns_cuda_error_before_launch(capi, monkeypatch):
+    """CSA2_INJECT_FAULT makes the named entry points fail as a failed launch
+    would (CSA2_ERR_CUDA), after the argument checks and before anything is
+    enqueued, and csa2_injected_faults counts it.  No GPU is involved: the
+    pointers are never dereferenced on the host."""
+    lib = capi.lib()
+    lib.csa2_injected_faults.restype = ctypes.c_int
+    c = capi.csa2_cache(*([16] * 10), 2, 1, 1, 2)
+    ws = capi.index_topk_workspace(2, 64, 4, 8)
+    w = capi.csa2_window(16, 16, 2, 0)
+
+    def topk():
+        return lib.csa2_index_topk(ctypes.byref(c), ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 8,
+                                   ctypes.c_void_p(16), None, ctypes.c_void_p(256), ctypes.c_size_t(ws), None)
+
+    def append():
+        return lib.csa2_window_append(ctypes.byref(w), ctypes.c_void_p(16), None)
+
+    n0 = lib.csa2_injected_faults()
+    monkeypatch.setenv("CSA2_INJECT_FAULT", "csa2_index_topk")
+    assert topk() == -4                                   # CSA2_ERR_CUDA, injected
+    assert lib.csa2_injected_faults() == n0 + 1
+    # an argument error still wins over the hook, and is not counted
+    assert lib.csa2_index_topk(ctypes.byref(c), ctypes.c_void_p(16), ctypes.c_void_p(16), 65, 8,
+                               ctypes.c_void_p(16), None, None, 0, None) == -1
+    assert lib.csa2_injected_faults() == n0 + 1
+    # other entry points are not listed: the window append is not injected
+    # (without a GPU it fails in CUDA itself, which the counter does not see)
+    append()
+    assert lib.csa2_injected_faults() == n0 + 1
+    monkeypatch.setenv("CSA2_INJECT_FAULT", "csa2_pack_cache,csa2_window_append")
+    assert append() == -4
+    assert lib.csa2_injected_faults() == n0 + 2
+    monkeypatch.setenv("CSA2_INJECT_FAULT", "*")
+    assert topk() == -4 and append() == -4
+    assert lib.csa2_injected_faults() == n0 + 4
+    monkeypatch.delenv("CSA2_INJECT_FAULT")
+    append()
+    assert lib.csa2_injected_faults() == n0 + 4

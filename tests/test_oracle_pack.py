@@ -231,3 +231,42 @@ def test_append_pending_slot(ref):
     assert np.array_equal(r1.mc[0, 5], c) and np.array_equal(r1.ms[0, 5], s)
     with pytest.raises(ValueError):
         ref.RefCache(1, 3, 2, Wm).append(0, x, g)
+
+
+def test_pack_scale_is_nearest_even_e4m3_of_amax_over_6(ref):
+    """The main scale byte is E4M3 round-to-nearest-even of fp32 amax / 6 (the
+    reading of "Le cache KV en FP4" in which the scale is the plain NVFP4-style
+    nearest value): pinned at every exact midpoint between two adjacent positive
+    E4M3 values, one fp32 ulp either side of it, and on the values themselves,
+    against the library float8 cast, independently of the GPU path."""
+    import torch
+    rng = np.random.default_rng(11)
+    vals = np.array([ref.e4m3_value(c) for c in range(0x7F)], np.float64)  # 0 .. 448
+    amaxes = []
+    for k in range(1, 0x7E):
+        lo, hi = vals[k], vals[k + 1]
+        for target in (lo, (lo + hi) / 2):
+            a = np.float32(target * 6.0)  # exact: few significant bits
+            assert float(a) == target * 6.0
+            amaxes += [a, np.nextafter(a, np.float32(np.inf)), np.nextafter(a, np.float32(0))]
+    amaxes = np.array(amaxes, np.float32)
+    amaxes = amaxes[(amaxes > 0) & (amaxes / np.float32(6) <= np.float32(448))]
+    want = torch.from_numpy(amaxes / np.float32(6)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for i0 in range(0, len(amaxes), 32):
+        blk = amaxes[i0:i0 + 32]
+        e = np.zeros(512, np.float32)
+        for j, a in enumerate(blk):
+            # one element carries +-amax, the others are strictly smaller
+            v = (rng.random(16) * 0.99 * a).astype(np.float32) * rng.choice([-1, 1], 16)
+            v[rng.integers(0, 16)] = a * rng.choice([-1, 1])
+            e[16 * j:16 * j + 16] = v
+        _, scales = ref.pack_main(e)
+        assert np.array_equal(scales[:len(blk)], want[i0:i0 + 32])
+    # the midpoints themselves went to the even code (ties-to-even, not round-up)
+    mids = np.array([np.float32((vals[k] + vals[k + 1]) / 2 * 6) for k in range(1, 0x7E)], np.float32)
+    e = np.zeros(512, np.float32)
+    for j in range(32):
+        e[16 * j] = mids[j]
+    _, scales = ref.pack_main(e)
+    for j in range(32):
+        assert scales[j] % 2 == 0
