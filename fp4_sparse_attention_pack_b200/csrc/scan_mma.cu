@@ -15,38 +15,43 @@
 // (two MMAs of K = 64 each).  The epilogue applies ReLU, the head weights and
 // the head sum, one thread per (entry row, problem).
 //
-// Persistent, warp-specialised CTA (640 threads, one CTA per SM):
-//   warps 0, 19  producers: TMA tile loads of the keys (one 64-entry page per
-//           box, 64-byte swizzle) and bulk copies of their E8M0 scales into an
-//           8-stage ring, the two warps taking alternate tiles; warp 0 also
-//           loads per work item the query tiles, scales and head weights of
-//           every problem of the subset (double-buffered).  Keys stream with an
-//           L2 evict-first policy.  Copies are issued by several lanes at once
-//           (a lane per page, per problem or per pool block): issued one by one
-//           from a single lane of a single warp, they set the pace of the whole
-//           pipeline when a subset holds one problem.
-//   warp 1  MMA issuer: per tile issues one MMA pass per
-//           problem pair into one of three TMEM accumulators (pass p into
-//           p % 3), committing each pass to its epilogue group.  Its only
-//           commits are those: the epilogue warp that sees a tile's last pass
-//           complete hands the key stage back to the producer, and the
-//           epilogue's arrivals after an item's last pass free the query
-//           buffer.  Three accumulators let the next pass run while both
-//           groups drain theirs.
+// A pass costs the tensor core 128 cycles and the epilogue's ReLU, weight and
+// sum over its 16,384 accumulators about twice that on the CUDA cores.  The
+// pass rate is bound by the hand-off between the two: measured on this GPU,
+// the commit of a pass becomes visible to a waiting warp ~600 cycles after the
+// MMAs were issued, so with three 128-column accumulators (what TMEM holds
+// beside the scale factors) and the epilogue's TMEM loads in the loop, a pass
+// costs ~300-450 cycles even with an empty epilogue.  Two alternating
+// epilogue groups keep the loads of one pass off the critical path of the next.
+//
+// Persistent, warp-specialised CTA (576 threads, one CTA per SM):
+//   warp 0  producer: decodes the CTA's work items (the only warp that reads the
+//           item tables among the kernel parameters) into a descriptor in shared
+//           memory per query buffer; per item the query tiles, query scales and
+//           head weights of every problem of the subset (double-buffered), per
+//           tile the key codes by TMA (one 64-entry page per box, 64-byte
+//           swizzle) and their E8M0 scales by bulk copy into an 8-stage ring.
+//           Keys stream with an L2 evict-first policy.  Tile copies are issued by
+//           one lane with warp-uniform operands.
+//   warp 1  MMA issuer: rearranges each stage's and each item's E8M0 scales into
+//           the 32x128-bit layout tcgen05.cp reads and copies them into TMEM, then
+//           issues one MMA pass per problem pair into one of three TMEM
+//           accumulators (pass p into p % 3), each pass committed to its
+//           accumulator's barrier; after a tile's passes a commit hands the key
+//           stage back to the producer, after an item's a commit releases the
+//           query buffer.  Copies and MMAs of one thread run in issue order, so
+//           no barrier separates a scale copy from the MMAs that read it.
 //   warps 2-17 epilogue, two groups of eight; group g drains the passes p with
-//           p % 2 == g.  Warp w of a group reads TMEM lane quadrant
-//           w % 4 and problem (w / 4) % 2 of the pass: tcgen05.ld of the 64 head
-//           columns of its entry, ReLU, weight, sum, one score store.
-//           A subset that scans a pool (hierarchical indexer) instead gathers
-//           each tile as 16 boxes of 8 rows, one per pool block, each into its
-//           own 512-byte slot, so the swizzled layout is that of a whole page.
-//   warp 18 scale warp: rearranges the E8M0 scales that landed in shared memory
-//           into the 32x128-bit layout tcgen05.cp reads (per item for the
-//           queries, per stage for the keys), copies them into TMEM and commits
-//           the copies to the ready barriers the MMA issuer waits on, keeping
-//           the transposition, its proxy fence and the copies off the issuer's
-//           path (one tcgen05 instruction costs the issuing warp about a hundred
-//           cycles).
+//           p % 2 == g.  Warp w of a group reads TMEM lane quadrant w % 4 and
+//           problem (w / 4) % 2 of the pass: two tcgen05.ld of 32 head columns
+//           each (the accumulator is released after the second), ReLU, weight,
+//           sum, one coalesced score store per 32 entries.  The ReLU is x + |x|
+//           (exactly twice max(x, 0), halved once at the end) on the FMA pipe:
+//           fmaxf would fill the half-rate ALU pipe, and busy ALU warps delay
+//           the tcgen05 instructions of the MMA warp on the same sub-partition.
+// A subset that scans a pool (hierarchical indexer) gathers each tile as 16
+// boxes of 8 rows, one per pool block, each into its own 512-byte slot, so the
+// swizzled layout is that of a whole page.
 // Every wait is bounded; a timeout sets CSA2_DEVERR_TIMEOUT in the problem's
 // status word and the CTA drains and exits.
 #include <cuda.h>
@@ -72,12 +77,11 @@ constexpr int kMaxPasses = kMaxSub / kPass;
 constexpr int kStages = 8;
 constexpr int kTile = 128;        // entries per MMA tile (MMA M)
 constexpr int kMaxChunk = 16;     // tiles per work item at most (32 pages: one per producer lane)
-constexpr int kGroups = 2;        // epilogue groups
-constexpr int kAcc = 3;           // TMEM accumulators: pass p lands in p % kAcc, group p % kGroups drains it
-constexpr int kEpiWarps = 8 * kGroups;
-constexpr int kSfWarp = 2 + kEpiWarps;
-constexpr int kProducer1Warp = kSfWarp + 1;  // second producer: the odd tiles
-constexpr int kThreads = 32 * (kProducer1Warp + 1);
+constexpr int kAcc = 3;           // TMEM accumulators: pass p lands in p % kAcc
+constexpr int kGroups = 2;        // epilogue groups: group g drains the passes p with p % 2 == g
+constexpr int kEpiWarps = 8 * kGroups;  // per group one per (TMEM lane quadrant, problem of the pass)
+constexpr int kEpi0 = 2;          // first epilogue warp
+constexpr int kThreads = 32 * (kEpi0 + kEpiWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = 0;                            // kAcc x 128 accumulator columns
 constexpr uint32_t kColSfa = 128 * kAcc;                   // kStages x 4 scale columns (keys)
@@ -105,6 +109,17 @@ struct MmaScanMaps {
     int n_items;
 };
 
+// A work item as the producer decodes it for the other roles (shared memory,
+// one per query buffer): the MMA and epilogue warps never touch the kernel
+// parameters inside their loops, whose dynamically indexed reads miss the
+// constant cache.
+struct ItemDesc {
+    int b, t0, t1, n;        // sequence, tile range, valid positions
+    int nprob;               // problems of the subset; 0 ends the CTA's work
+    uint32_t* status;        // status word of the cache
+    float* rows[kMaxSub];    // each problem's score row of sequence b
+};
+
 struct __align__(1024) Smem {
     uint8_t a[kStages][kTile * 64];          // key codes, 64B-swizzled rows
     uint8_t b[2][kMaxSub * kHeads * 64];     // query codes of the subset, 64B-swizzled rows
@@ -113,12 +128,12 @@ struct __align__(1024) Smem {
     uint8_t sfb_raw[2][kMaxSub * kHeads * 4];
     uint8_t sfb_tc[2][kMaxPasses][512];
     float w[2][kMaxSub][kHeads];
-    float* rows[2][kMaxSub];                 // score row of the item's sequence, per problem
-    int prow[2][kMaxChunk * 16];             // pool items, per producer: first physical key row of each slot
-    uint64_t full[kStages], empty[kStages], sfa_ready[kStages];
-    uint64_t bfull[2], bempty[2], sfb_ready[2];
+    ItemDesc desc[2];
+    int prow[kMaxChunk * 16];                // pool items: first physical key row of each slot
+    uint64_t full[kStages], empty[kStages];
+    uint64_t qfull[2], qempty[2];
     uint64_t tfull[kAcc], tempty[kAcc];
-    uint64_t drained, sdrained;
+    uint64_t drained;
     uint32_t tmem_base;
     int abort;
 };
@@ -129,6 +144,10 @@ struct Item {
     int s, b, t0, t1, n;
 };
 
+// Work item id -> (subset, sequence, tile range).  Every lane of the warp must
+// call it.  Lane 0's entry count is shuffled to the whole warp, so the
+// compiler knows every loop bound, ring index and copy operand derived from
+// the item is warp-uniform.
 __device__ __forceinline__ bool item_at(const ScanBatch& sb, const MmaScanMaps& mp, int id, Item& it) {
     int s = 0;
     while (s + 1 < mp.n_sub && id >= mp.sub[s + 1].item0) ++s;
@@ -138,15 +157,12 @@ __device__ __forceinline__ bool item_at(const ScanBatch& sb, const MmaScanMaps& 
     it.b = r / S.chunks;
     const int c = r - it.b * S.chunks;
     const ScanProblem& P0 = sb.p[S.prob[0]];
-    it.n = S.pool ? min(max(P0.pool_n[it.b], 0), kPoolBlock * P0.pool_blocks) : entries_of(P0.cache, it.b);
-    const int tiles = (it.n + kTile - 1) / kTile;
+    int n = S.pool ? min(max(P0.pool_n[it.b], 0), kPoolBlock * P0.pool_blocks) : entries_of(P0.cache, it.b);
+    n = __shfl_sync(0xffffffffu, n, 0);
+    const int tiles = (n + kTile - 1) / kTile;
+    it.n = n;
     it.t0 = c * S.chunk;
     it.t1 = min(it.t0 + S.chunk, tiles);
-    // Lane 0's values for the whole warp: the compiler then sees every loop
-    // bound and ring index derived from them as warp-uniform, so the tcgen05
-    // operands built from them need no per-lane handling at issue.
-    it.n = __shfl_sync(0xffffffffu, it.n, 0);
-    it.t1 = __shfl_sync(0xffffffffu, it.t1, 0);
     return it.t0 < it.t1;
 }
 
@@ -178,31 +194,51 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     return r;
 }
 
+// 2 max(x, 0), exactly: x + |x| is 2x or 0.  One add with an absolute-value
+// operand on the FMA pipe, where fmaxf would occupy the half-rate ALU pipe that
+// the MMA and producer warps need for their own instructions.
+__device__ __forceinline__ float relu2(float x) { return x + fabsf(x); }
+
+// acc += w[h] * 2 max(v[h], 0) over N heads: head h goes to fp32 chain h % 8
+// (four packed pairs).  The caller halves the fixed pairwise sum of the
+// chains at the end (exact), so the score equals the one formed with max(v, 0).
+template <int N>
+__device__ __forceinline__ void relu_weighted_acc(const float (&v)[N], const float* w, float2 (&acc2)[4]) {
+#pragma unroll
+    for (int h = 0; h < N; h += 8) {
+        const float4 wa = *reinterpret_cast<const float4*>(w + h);
+        const float4 wb = *reinterpret_cast<const float4*>(w + h + 4);
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = relu2(v[h + i]);
+        acc2[0] = fma2(make_float2(wa.x, wa.y), make_float2(x[0], x[1]), acc2[0]);
+        acc2[1] = fma2(make_float2(wa.z, wa.w), make_float2(x[2], x[3]), acc2[1]);
+        acc2[2] = fma2(make_float2(wb.x, wb.y), make_float2(x[4], x[5]), acc2[2]);
+        acc2[3] = fma2(make_float2(wb.z, wb.w), make_float2(x[6], x[7]), acc2[3]);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_scan_mma(const __grid_constant__ ScanBatch sb, const __grid_constant__ MmaScanMaps mp) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int batch = sb.p[0].cache.batch;
     const int n_items = mp.n_items;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 1);  // the epilogue warp that sees the tile's last pass complete
-            mbar_init(&sm.sfa_ready[s], 1);
+            mbar_init(&sm.empty[s], 1);  // the MMA warp's commit after the tile's last pass
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.bfull[i], 1);
-            mbar_init(&sm.bempty[i], kEpiWarps);  // after the item's last pass: its MMAs are done
-            mbar_init(&sm.sfb_ready[i], 1);
+            mbar_init(&sm.qfull[i], 1);
+            mbar_init(&sm.qempty[i], 1 + kEpiWarps);  // the MMA warp's commit + every epilogue warp
         }
         for (int a = 0; a < kAcc; ++a) {
             mbar_init(&sm.tfull[a], 1);
             mbar_init(&sm.tempty[a], 8);  // the eight warps of the group that drains it
         }
         mbar_init(&sm.drained, 1);
-        mbar_init(&sm.sdrained, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -210,149 +246,158 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tbase = __shfl_sync(0xffffffffu, sm.tmem_base, 0);  // warp-uniform (see item_at)
+    const uint32_t tbase = __shfl_sync(0xffffffffu, sm.tmem_base, 0);
 
-    if (warp == 0 || warp == kProducer1Warp) {
-        // ------------------------------------------------------------ producers
-        // Two warps walk the same items; the CTA's tiles are numbered in order (g)
-        // and producer pw loads the tiles with g % 2 == pw into stage g % kStages
-        // (kStages is even, so every use of a stage belongs to one producer).
-        // Producer 0 also loads each item's queries.  Lanes fetch the item's page
-        // ids (2 per tile, up to 32) in one round; barrier arms come from one
-        // elected lane, and the copies of a tile or an item are issued by several
-        // lanes at once.
-        const uint32_t pw = warp == 0 ? 0u : 1u;
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        const int batch = sb.p[0].cache.batch;
         const uint64_t pol_stream = policy_evict_first();
         const uint64_t pol_keep = policy_evict_last();
-        if (lane == 0 && pw == 0) prefetch_tmap(&mp.queries);
+        if (lane == 0) prefetch_tmap(&mp.queries);
         uint32_t g = 0, bslot = 0, bphase = 0;
         uint32_t issued = 0, issued_par = 0;  // per stage: a copy was issued, and its phase
-        for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
+        bool stop = false;
+        for (int id = blockIdx.x; id < n_items && !stop; id += gridDim.x) {
             Item it;
             if (!item_at(sb, mp, id, it)) continue;
             const ScanSub& S = mp.sub[it.s];
-            const CacheView& c = sb.p[S.prob[0]].cache;
+            const int nprob = S.n, src = S.src, pool = S.pool;
+            const ScanProblem& P0 = sb.p[S.prob[0]];
+            const int32_t* page_table = P0.cache.page_table + (int64_t)it.b * P0.cache.max_pages;
+            const int max_pages = P0.cache.max_pages, num_pages = P0.cache.num_pages;
+            const uint8_t* idx_scales = P0.cache.idx_scales;
+            uint32_t* status = P0.cache.status;
+            // the item's page ids, one per lane (two pages a tile, at most 32)
             const int used_pages = (it.n + PAGE - 1) / PAGE;
-            const int li = 2 * it.t0 + lane;  // logical page this lane looks up
+            const int li = 2 * it.t0 + lane;
             int my_pg = -1;
-            if (!S.pool && lane < 2 * (it.t1 - it.t0) && li < used_pages) {
-                const int pp = c.page_table[(int64_t)it.b * c.max_pages + li];
-                if (pp >= 0 && pp < c.num_pages)
+            if (!pool && lane < 2 * (it.t1 - it.t0) && li < used_pages) {
+                const int pp = page_table[li];
+                if (pp >= 0 && pp < num_pages)
                     my_pg = pp;
                 else
-                    atomicOr(c.status, CSA2_DEVERR_PAGE);
+                    atomicOr(status, CSA2_DEVERR_PAGE);
             }
-            bool stop = false;
-            if (pw != 0) {
-                // queries are producer 0's
-            } else if (!mbar_wait_warp(&sm.bempty[bslot], bphase ^ 1)) {
-                if (lane == 0) raise_abort(sm, c.status);
-                stop = true;
-            } else {
-                if (lane < S.n) sm.rows[bslot][lane] = sb.p[S.prob[lane]].scores + (int64_t)it.b * sb.score_stride;
-                __syncwarp();
-                mbar_expect_tx_w(&sm.bfull[bslot], S.n * (kHeads * 64 + kHeads * 4 + kHeads * 4));
-                __syncwarp();
-                // lane j issues problem j's copies: one warp instruction per kind of copy
-                if (lane < S.n) {
-                    const int p = S.prob[lane];
-                    const int64_t qrow = ((int64_t)p * batch + it.b) * kHeads;
-                    tma_load_2d(sm.b[bslot] + lane * kHeads * 64, &mp.queries, 0, (int)qrow, &sm.bfull[bslot], pol_keep);
-                    bulk_load(sm.sfb_raw[bslot] + lane * kHeads * 4, sb.qs + qrow * ISB, kHeads * 4, &sm.bfull[bslot],
-                              pol_keep);
-                    bulk_load(sm.w[bslot][lane], sb.p[p].w + (int64_t)it.b * kHeads, kHeads * 4, &sm.bfull[bslot],
-                              pol_keep);
-                }
-                __syncwarp();
+            // the query buffer (and its item descriptor) is free once the item two
+            // back is done: its MMAs completed and every epilogue warp left it
+            if (!mbar_wait_warp(&sm.qempty[bslot], bphase ^ 1)) {
+                if (lane == 0) raise_abort(sm, status);
+                break;
             }
+            ItemDesc& D = sm.desc[bslot];
+            if (lane < nprob) D.rows[lane] = sb.p[S.prob[lane]].scores + (int64_t)it.b * sb.score_stride;
+            if (lane == 0) {
+                D.b = it.b;
+                D.t0 = it.t0;
+                D.t1 = it.t1;
+                D.n = it.n;
+                D.nprob = nprob;
+                D.status = status;
+            }
+            __syncwarp();
+            // queries, scales and head weights of the subset's problems (the
+            // arrival also publishes the descriptor)
+            mbar_expect_tx_w(&sm.qfull[bslot], nprob * (kHeads * 64 + kHeads * 4 + kHeads * 4));
+            __syncwarp();
+            if (lane < nprob) {  // lane j: problem j's three copies
+                const int p = S.prob[lane];
+                const int64_t qrow = ((int64_t)p * batch + it.b) * kHeads;
+                tma_load_2d(sm.b[bslot] + lane * kHeads * 64, &mp.queries, 0, (int)qrow, &sm.qfull[bslot], pol_keep);
+                bulk_load(sm.sfb_raw[bslot] + lane * kHeads * 4, sb.qs + qrow * ISB, kHeads * 4, &sm.qfull[bslot],
+                          pol_keep);
+                bulk_load(sm.w[bslot][lane], sb.p[p].w + (int64_t)it.b * kHeads, kHeads * 4, &sm.qfull[bslot],
+                          pol_keep);
+            }
+            __syncwarp();
             if (++bslot == 2) bslot = 0, bphase ^= 1;
-            const CUtensorMap* kmap = &mp.keys[S.src];
-            if (S.pool) {
+            const CUtensorMap* kmap = pool ? &mp.keys8[src] : &mp.keys[src];
+            if (pool) {
                 // physical first row of every pool block of the item (positions
                 // below it.n are valid, so their blocks lie below n_entries)
-                const ScanProblem& P0 = sb.p[S.prob[0]];
+                const int32_t* pool_ids = P0.pool + (int64_t)it.b * P0.pool_blocks;
                 const int slots = (it.n + kPoolBlock - 1) / kPoolBlock;
-                const int n_slot = 16 * (it.t1 - it.t0);  // <= 32 * kSlotsPerLane
+                const int n_slot = 16 * (it.t1 - it.t0);
                 constexpr int kSlotsPerLane = kMaxChunk * 16 / 32;
                 __syncwarp();  // the previous item's reads of prow are done
-                // all of a lane's block ids, then all their page ids: two rounds of
-                // independent loads instead of a chain of dependent pairs
                 int blk[kSlotsPerLane], pg[kSlotsPerLane];
 #pragma unroll
                 for (int j = 0; j < kSlotsPerLane; ++j) {
                     const int i = lane + 32 * j, slot = 16 * it.t0 + i;
-                    blk[j] = (i < n_slot && slot < slots) ? P0.pool[(int64_t)it.b * P0.pool_blocks + slot] : -1;
-                    if (blk[j] >= c.max_pages * (PAGE / kPoolBlock)) blk[j] = -1;  // never past the table
+                    blk[j] = (i < n_slot && slot < slots) ? pool_ids[slot] : -1;
+                    if (blk[j] >= max_pages * (PAGE / kPoolBlock)) blk[j] = -1;  // never past the table
                 }
 #pragma unroll
-                for (int j = 0; j < kSlotsPerLane; ++j)
-                    pg[j] = blk[j] >= 0 ? c.page_table[(int64_t)it.b * c.max_pages + kPoolBlock * blk[j] / PAGE] : -1;
+                for (int j = 0; j < kSlotsPerLane; ++j) pg[j] = blk[j] >= 0 ? page_table[kPoolBlock * blk[j] / PAGE] : -1;
 #pragma unroll
                 for (int j = 0; j < kSlotsPerLane; ++j) {
                     const int i = lane + 32 * j;
                     if (i >= n_slot) continue;
                     int r = -1;
                     if (blk[j] >= 0) {
-                        if (pg[j] >= 0 && pg[j] < c.num_pages)
+                        if (pg[j] >= 0 && pg[j] < num_pages)
                             r = pg[j] * PAGE + kPoolBlock * blk[j] % PAGE;
                         else
-                            atomicOr(c.status, CSA2_DEVERR_PAGE);
+                            atomicOr(status, CSA2_DEVERR_PAGE);
                     }
-                    sm.prow[pw][i] = r;
+                    sm.prow[i] = r;
                 }
                 __syncwarp();
             }
-            for (int t = it.t0; t < it.t1 && !stop; ++t, ++g) {
-                if ((g & 1u) != pw) continue;
+            for (int t = it.t0; t < it.t1; ++t, ++g) {
                 const uint32_t stage = g % kStages, sphase = (g / kStages) & 1u;
-                const int pg0 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0));
-                const int pg1 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0) + 1);
-                const int prow = S.pool && lane < 16 ? sm.prow[pw][16 * (t - it.t0) + lane] : -1;
-                const unsigned have = __ballot_sync(0xffffffffu, prow >= 0);
                 if (!mbar_wait_warp(&sm.empty[stage], sphase ^ 1)) {
-                    if (lane == 0) raise_abort(sm, c.status);
+                    if (lane == 0) raise_abort(sm, status);
                     stop = true;
                     break;
                 }
-                if (S.pool) {
+                if (pool) {
+                    const int prow = lane < 16 ? sm.prow[16 * (t - it.t0) + lane] : -1;
+                    const unsigned have = __ballot_sync(0xffffffffu, prow >= 0);
                     if (have == 0) {
                         mbar_arrive_w(&sm.full[stage]);
                     } else {
                         mbar_expect_tx_w(&sm.full[stage], __popc(have) * kPoolBlock * (ICB + ISB));
                         __syncwarp();
                         if (prow >= 0) {
-                            tma_load_2d(sm.a[stage] + lane * kPoolBlock * ICB, &mp.keys8[S.src], 0, prow,
-                                        &sm.full[stage], pol_stream);
-                            bulk_load(sm.sfa_raw[stage] + lane * kPoolBlock * ISB, c.idx_scales + (int64_t)prow * ISB,
+                            tma_load_2d(sm.a[stage] + lane * kPoolBlock * ICB, kmap, 0, prow, &sm.full[stage],
+                                        pol_stream);
+                            bulk_load(sm.sfa_raw[stage] + lane * kPoolBlock * ISB, idx_scales + (int64_t)prow * ISB,
                                       kPoolBlock * ISB, &sm.full[stage], pol_stream);
                         }
+                        __syncwarp();
                     }
-                    issued |= 1u << stage;
-                    issued_par = (issued_par & ~(1u << stage)) | (sphase << stage);
-                    continue;
-                }
-                const uint32_t bytes = (pg0 >= 0 ? PAGE * (ICB + ISB) : 0) + (pg1 >= 0 ? PAGE * (ICB + ISB) : 0);
-                if (bytes == 0) {
-                    mbar_arrive_w(&sm.full[stage]);
                 } else {
-                    mbar_expect_tx_w(&sm.full[stage], bytes);
-                    __syncwarp();
-                    // lanes 0, 1 load the two pages' key codes, lanes 2, 3 their scales
-                    const int h = lane & 1;
-                    const int pg = h ? pg1 : pg0;
-                    if (lane < 4 && pg >= 0) {
-                        if (lane < 2)
-                            tma_load_2d(sm.a[stage] + h * PAGE * ICB, kmap, 0, pg * PAGE, &sm.full[stage], pol_stream);
-                        else
-                            bulk_load(sm.sfa_raw[stage] + h * PAGE * ISB, c.idx_scales + (int64_t)pg * PAGE * ISB,
+                    const int pg0 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0));
+                    const int pg1 = __shfl_sync(0xffffffffu, my_pg, 2 * (t - it.t0) + 1);
+                    const uint32_t bytes = (pg0 >= 0 ? PAGE * (ICB + ISB) : 0) + (pg1 >= 0 ? PAGE * (ICB + ISB) : 0);
+                    if (bytes == 0) {
+                        mbar_arrive_w(&sm.full[stage]);
+                    } else if (lane == 0) {
+                        mbar_expect_tx(&sm.full[stage], bytes);
+                        if (pg0 >= 0) {
+                            tma_load_2d(sm.a[stage], kmap, 0, pg0 * PAGE, &sm.full[stage], pol_stream);
+                            bulk_load(sm.sfa_raw[stage], idx_scales + (int64_t)pg0 * PAGE * ISB, PAGE * ISB,
+                                      &sm.full[stage], pol_stream);
+                        }
+                        if (pg1 >= 0) {
+                            tma_load_2d(sm.a[stage] + PAGE * ICB, kmap, 0, pg1 * PAGE, &sm.full[stage], pol_stream);
+                            bulk_load(sm.sfa_raw[stage] + PAGE * ISB, idx_scales + (int64_t)pg1 * PAGE * ISB,
                                       PAGE * ISB, &sm.full[stage], pol_stream);
+                        }
                     }
                     __syncwarp();
                 }
                 issued |= 1u << stage;
                 issued_par = (issued_par & ~(1u << stage)) | (sphase << stage);
             }
-            if (stop) break;
+            stop = stop || __any_sync(0xffffffffu, aborted(sm));
+        }
+        // the end of the CTA's work: a descriptor with no problems
+        if (!stop && mbar_wait_warp(&sm.qempty[bslot], bphase ^ 1)) {
+            if (lane == 0) {
+                sm.desc[bslot].nprob = 0;
+                mbar_arrive(&sm.qfull[bslot]);
+            }
         }
         // never leave with copies in flight
         if (lane == 0)
@@ -360,26 +405,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if ((issued >> s) & 1u) (void)mbar_wait(&sm.full[s], (issued_par >> s) & 1u);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0, acc = 0, aphase = 0;
-        for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
-            Item it;
-            if (!item_at(sb, mp, id, it)) continue;
-            const ScanSub& S = mp.sub[it.s];
-            uint32_t* status = sb.p[S.prob[0]].cache.status;
-            const int passes = (S.n + kPass - 1) / kPass;
-            // the query scales of the item are in TMEM once sfb_ready completes
-            if (!mbar_wait_warp(&sm.sfb_ready[bslot], bphase)) { raise_abort(sm, status); break; }
+        uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0, pass_no = 0;
+        uint32_t* status = sb.p[0].cache.status;
+        while (true) {
+            if (!mbar_wait_warp(&sm.qfull[bslot], bphase)) {
+                if (lane == 0) raise_abort(sm, status);
+                break;
+            }
+            const ItemDesc& D = sm.desc[bslot];
+            // lane 0's copies: warp-uniform to the compiler, so the loops below
+            // and the tcgen05 operands derived from their counters need no
+            // per-lane handling at issue
+            const int nprob = __shfl_sync(0xffffffffu, D.nprob, 0);
+            const int t0 = __shfl_sync(0xffffffffu, D.t0, 0), t1 = __shfl_sync(0xffffffffu, D.t1, 0);
+            if (nprob == 0) break;
+            status = D.status;
+            const int passes = (nprob + kPass - 1) / kPass;
+            // the item's query scales into TMEM (the columns' previous reader, the
+            // item two back, has completed: its commit preceded this buffer's reload)
+            tc_fence_after();
+            for (int k = 0; k < passes; ++k) scales_to_tc(sm.sfb_raw[bslot] + k * 512, sm.sfb_tc[bslot][k], lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            for (int k = 0; k < passes; ++k)
+                tc_cp_32x128b_x4_w(tbase + kColSfb + (bslot * kMaxPasses + k) * 4,
+                                   smem_desc(sm.sfb_tc[bslot][k], 16, 128, kLayoutNone));
             bool stop = false;
-            for (int t = it.t0; t < it.t1; ++t) {
-                // ... and the stage's key scales once sfa_ready completes
-                if (!mbar_wait_warp(&sm.sfa_ready[stage], sphase)) { raise_abort(sm, status); stop = true; break; }
-                const uint32_t sfa = tbase + kColSfa + 4 * stage;
+            for (int t = t0; t < t1; ++t) {
+                if (!mbar_wait_warp(&sm.full[stage], sphase)) {
+                    if (lane == 0) raise_abort(sm, status);
+                    stop = true;
+                    break;
+                }
+                // the stage's key scales into TMEM (their previous reader, the tile
+                // eight back, completed before the producer could refill the stage)
                 tc_fence_after();
+                scales_to_tc(sm.sfa_raw[stage], sm.sfa_tc[stage], lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                const uint32_t sfa = tbase + kColSfa + 4 * stage;
+                tc_cp_32x128b_x4_w(sfa, smem_desc(sm.sfa_tc[stage], 16, 128, kLayoutNone));
                 const uint64_t adesc = smem_desc(sm.a[stage], 16, 512, kLayoutSw64);
-                for (int k = 0; k < passes; ++k) {
-                    if (!mbar_wait_warp(&sm.tempty[acc], aphase ^ 1)) { raise_abort(sm, status); stop = true; break; }
+                for (int k = 0; k < passes; ++k, ++pass_no) {
+                    const uint32_t acc = pass_no % kAcc;
+                    if (!mbar_wait_warp(&sm.tempty[acc], ((pass_no / kAcc) & 1u) ^ 1u)) {
+                        if (lane == 0) raise_abort(sm, status);
+                        stop = true;
+                        break;
+                    }
                     tc_fence_after();
-                    const uint32_t n_rows = (uint32_t)min(kPass, S.n - kPass * k) * kHeads;
+                    const uint32_t n_rows = (uint32_t)min(kPass, nprob - kPass * k) * kHeads;
                     const uint32_t sfb = tbase + kColSfb + (bslot * kMaxPasses + k) * 4;
                     const uint32_t d = tbase + kColAcc + 128 * acc;
                     const uint64_t bdesc = smem_desc(sm.b[bslot] + k * kPass * kHeads * 64, 16, 512, kLayoutSw64);
@@ -387,80 +462,79 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_mma_mxf4_w(d, adesc, bdesc, idesc_mxf4(n_rows, 0, 0), sfa, sfb, 0u);
                     tc_mma_mxf4_w(d, adesc + 2, bdesc + 2, idesc_mxf4(n_rows, 2, 2), sfa, sfb, 1u);
                     tc_commit_w(&sm.tfull[acc]);
-                    if (++acc == kAcc) acc = 0, aphase ^= 1;
                 }
                 if (stop) break;
+                tc_commit_w(&sm.empty[stage]);  // the stage is free once these MMAs complete
                 if (++stage == kStages) stage = 0, sphase ^= 1;
             }
-            if (++bslot == 2) bslot = 0, bphase ^= 1;
             if (stop) break;
+            tc_commit_w(&sm.qempty[bslot]);  // the item's MMAs no longer read its queries
+            if (++bslot == 2) bslot = 0, bphase ^= 1;
         }
         // every tcgen05 operation of this thread has completed before TMEM is freed
         tc_commit_w(&sm.drained);
         (void)mbar_wait_warp(&sm.drained, 0);
-    } else if (warp < kSfWarp) {
+    } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - 2;
-        const int grp = ew >> 3;
-        const int jp = (ew >> 2) & 1;     // problem of the pass this warp reads
-        const int quad = warp & 3;        // TMEM lane quadrant of this warp
+        // Two groups of eight warps; group g drains the passes p with p % 2 == g.
+        // Warp w of a group reads TMEM lane quadrant w % 4 (entries 32 (w % 4) ..
+        // + 31 of the tile) and problem (w / 4) % 2 of the pass: two loads of 32
+        // head columns (the accumulator is released after the second), ReLU,
+        // weight and head sum, one coalesced store per 32 entries.
+        const int ew = warp - kEpi0;
+        const uint32_t grp = (uint32_t)(ew >> 3);
+        const int jp = (ew >> 2) & 1;
+        const int quad = warp & 3;
         const int row = quad * 32 + lane;
-        uint32_t bslot = 0, bphase = 0, pass_no = 0, stage = 0;
-        for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
-            Item it;
-            if (!item_at(sb, mp, id, it)) continue;
-            const ScanSub& S = mp.sub[it.s];
-            const int passes = (S.n + kPass - 1) / kPass;
-            uint32_t* status = sb.p[S.prob[0]].cache.status;
-            if (!mbar_wait_warp(&sm.bfull[bslot], bphase)) { raise_abort(sm, status); break; }
+        const uint32_t tlane = tbase + ((uint32_t)(quad * 32) << 16) + kColAcc + 64 * jp;
+        uint32_t bslot = 0, bphase = 0, pass_no = 0;
+        uint32_t* status = sb.p[0].cache.status;
+        while (true) {
+            if (!mbar_wait_warp(&sm.qfull[bslot], bphase)) {
+                if (lane == 0) raise_abort(sm, status);
+                break;
+            }
+            const ItemDesc& D = sm.desc[bslot];
+            const int nprob = __shfl_sync(0xffffffffu, D.nprob, 0);  // warp-uniform, as in the MMA warp
+            const int t0 = __shfl_sync(0xffffffffu, D.t0, 0), t1 = __shfl_sync(0xffffffffu, D.t1, 0);
+            const int n = D.n;
+            if (nprob == 0) break;
+            status = D.status;
+            const int passes = (nprob + kPass - 1) / kPass;
             bool stop = false;
-            for (int t = it.t0; t < it.t1 && !stop; ++t, stage = stage + 1 == kStages ? 0 : stage + 1) {
+            for (int t = t0; t < t1 && !stop; ++t) {
+                const int e = t * kTile + row;
                 for (int k = 0; k < passes; ++k, ++pass_no) {
-                    if ((int)(pass_no % kGroups) != grp) continue;
-                    const int acc = (int)(pass_no % kAcc);
+                    if (pass_no % kGroups != grp) continue;
+                    const uint32_t acc = pass_no % kAcc;
                     if (!mbar_wait_warp(&sm.tfull[acc], (pass_no / kAcc) & 1u)) {
-                        raise_abort(sm, status);
+                        if (lane == 0) raise_abort(sm, status);
                         stop = true;
                         break;
                     }
-                    // the tile's last pass has completed, and every MMA before it:
-                    // its key stage goes back to the producer
-                    if (k == passes - 1 && (ew & 7) == 0 && lane == 0) mbar_arrive(&sm.empty[stage]);
                     tc_fence_after();
                     const int j = kPass * k + jp;
-                    if (j < S.n) {
-                        const uint32_t taddr = tbase + ((uint32_t)(quad * 32) << 16) + kColAcc + 128 * acc + 64 * jp;
+                    if (j < nprob) {
                         const float* w = sm.w[bslot][j];
-                        float2 acc2[4];  // eight chains: heads h = 8i + c go to chain c
+                        float2 acc2[4];
 #pragma unroll
                         for (int c = 0; c < 4; ++c) acc2[c] = make_float2(0.0f, 0.0f);
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            float v[32];
-                            tmem_ld_32x32b_x32(taddr + 32 * half, v);
-                            if (half == 1) {
-                                tc_fence_before();
-                                __syncwarp();
-                                if (lane == 0) mbar_arrive(&sm.tempty[acc]);
-                            }
-#pragma unroll
-                            for (int h = 0; h < 32; h += 8) {
-                                const float4 wa = *reinterpret_cast<const float4*>(w + 32 * half + h);
-                                const float4 wb = *reinterpret_cast<const float4*>(w + 32 * half + h + 4);
-                                acc2[0] = fma2(make_float2(wa.x, wa.y), make_float2(fmaxf(v[h], 0.0f), fmaxf(v[h + 1], 0.0f)),
-                                               acc2[0]);
-                                acc2[1] = fma2(make_float2(wa.z, wa.w),
-                                               make_float2(fmaxf(v[h + 2], 0.0f), fmaxf(v[h + 3], 0.0f)), acc2[1]);
-                                acc2[2] = fma2(make_float2(wb.x, wb.y),
-                                               make_float2(fmaxf(v[h + 4], 0.0f), fmaxf(v[h + 5], 0.0f)), acc2[2]);
-                                acc2[3] = fma2(make_float2(wb.z, wb.w),
-                                               make_float2(fmaxf(v[h + 6], 0.0f), fmaxf(v[h + 7], 0.0f)), acc2[3]);
-                            }
+                        {
+                            float v0[32];
+                            tmem_ld_32x32b_x32(tlane + 128 * acc, v0);
+                            relu_weighted_acc(v0, w, acc2);
                         }
-                        const float s = ((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) +
-                                        ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y));
-                        const int e = t * kTile + row;
-                        if (e < it.n) sm.rows[bslot][j][e] = s;
+                        {
+                            float v1[32];
+                            tmem_ld_32x32b_x32(tlane + 128 * acc + 32, v1);
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&sm.tempty[acc]);
+                            relu_weighted_acc(v1, w + 32, acc2);
+                        }
+                        const float s = 0.5f * (((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) +
+                                                ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y)));
+                        if (e < n) D.rows[j][e] = s;
                     } else {
                         tc_fence_before();
                         __syncwarp();
@@ -469,53 +543,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.bempty[bslot]);
+            if (lane == 0) mbar_arrive(&sm.qempty[bslot]);
             if (++bslot == 2) bslot = 0, bphase ^= 1;
             if (stop) break;
         }
-    } else {
-        // ------------------------------------------------------------ scale warp
-        uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0;
-        for (int id = blockIdx.x; id < n_items && !__any_sync(0xffffffffu, aborted(sm)); id += gridDim.x) {
-            Item it;
-            if (!item_at(sb, mp, id, it)) continue;
-            const ScanSub& S = mp.sub[it.s];
-            uint32_t* status = sb.p[S.prob[0]].cache.status;
-            const int passes = (S.n + kPass - 1) / kPass;
-            if (!mbar_wait_warp(&sm.bfull[bslot], bphase)) { if (lane == 0) raise_abort(sm, status); break; }
-            // bfull implies the MMAs of the item two back, which read these TMEM
-            // columns, have completed (bempty follows its last pass's completion)
-            tc_fence_after();
-            for (int k = 0; k < passes; ++k) scales_to_tc(sm.sfb_raw[bslot] + k * 512, sm.sfb_tc[bslot][k], lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-            for (int k = 0; k < passes; ++k)
-                tc_cp_32x128b_x4_w(tbase + kColSfb + (bslot * kMaxPasses + k) * 4,
-                                   smem_desc(sm.sfb_tc[bslot][k], 16, 128, kLayoutNone));
-            tc_commit_w(&sm.sfb_ready[bslot]);
-            if (++bslot == 2) bslot = 0, bphase ^= 1;
-            bool stop = false;
-            for (int t = it.t0; t < it.t1; ++t) {
-                if (!mbar_wait_warp(&sm.full[stage], sphase)) {
-                    if (lane == 0) raise_abort(sm, status);
-                    stop = true;
-                    break;
-                }
-                // full implies the MMAs that last read this stage's scale columns
-                // have completed (the stage's empty arrival follows them)
-                tc_fence_after();
-                scales_to_tc(sm.sfa_raw[stage], sm.sfa_tc[stage], lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-                tc_cp_32x128b_x4_w(tbase + kColSfa + 4 * stage, smem_desc(sm.sfa_tc[stage], 16, 128, kLayoutNone));
-                tc_commit_w(&sm.sfa_ready[stage]);
-                if (++stage == kStages) stage = 0, sphase ^= 1;
-            }
-            if (stop) break;
-        }
-        // every scale copy of this warp has completed before TMEM is freed
-        tc_commit_w(&sm.sdrained);
-        (void)mbar_wait_warp(&sm.sdrained, 0);
     }
 
     tc_fence_before();
