@@ -9,9 +9,10 @@
 // (pool build: the winners are block ids).
 //
 // One CTA of 512 threads per (problem, sequence):
-//   1. Threshold guess: 2,048 strided samples of the row; an exact radix select
-//      in shared memory finds the sample key ranked ~2K * 2048 / n, so that
-//      about 2K of the n scores lie at or above it.
+//   1. Threshold guess: 2,048 samples of the row (256 evenly spaced runs of 8
+//      consecutive scores); a radix select in shared memory finds the leading
+//      16 bits of the sample key ranked ~2K * 2048 / n, so that about 2K of the
+//      n scores lie at or above it.
 //   2. One pass over the row compacts every score at or above the guess, in
 //      index order, into shared memory (at most kCap).  If fewer than K or more
 //      than kCap qualify, the CTA falls back to an exact radix select over the
@@ -33,6 +34,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kSamples = 2048;
 constexpr int kCap = 4096;  // candidates kept in shared memory (the guess targets about 2K + 1 %)
 constexpr int kRun = 8;   // contiguous scores per thread per pass
+constexpr int kSampleRun = 8;  // consecutive scores per sample run (one 32-byte sector)
 
 struct TopkSmem {
     uint32_t key[kCap];
@@ -83,12 +85,14 @@ __device__ __forceinline__ void hist_add(int* hist, uint32_t d) {
 
 // Exact radix select: the k-th largest key among key(i), i < cnt (k <= cnt), and
 // how many keys equal to it belong to the top k.  8-bit digits, MSB first.
+// With passes < 4 the result is the k-th largest key's leading 8 * passes bits
+// with the rest zero, a lower bound of it (need is then meaningless).
 template <class KeyAt>
-__device__ void radix_select(KeyAt key_at, int cnt, int k, TopkSmem& sm, uint32_t* kth, int* need) {
+__device__ void radix_select(KeyAt key_at, int cnt, int k, TopkSmem& sm, uint32_t* kth, int* need, int passes = 4) {
     uint32_t prefix = 0, mask = 0;
     int remaining = k;
     const int tid = threadIdx.x;
-    for (int pass = 0; pass < 4; ++pass) {
+    for (int pass = 0; pass < passes; ++pass) {
         const int sh = 24 - 8 * pass;
         if (tid < 256) sm.hist[tid] = 0;
         __syncthreads();
@@ -187,17 +191,25 @@ __global__ void __launch_bounds__(kThreads, 4) k_topk(const __grid_constant__ Sc
         return;
     }
 
-    // 1. threshold guess from strided samples (all scores qualify when they fit):
+    // 1. threshold guess from sampled scores (all scores qualify when they fit):
     // about 2K candidates, at most halfway from K to kCap
     uint32_t guess = 0;
     if (n > kCap && K < kCap) {
-        for (int i = tid; i < kSamples; i += kThreads)
-            sm.key[i] = f32_order_key(row[(int64_t)i * n / kSamples]);
+        // 256 evenly spaced runs of 8 consecutive scores, one 32-byte sector
+        // each: single samples every n / 2048 scores would touch every cache
+        // line of a 65,536-entry row and cost the memory traffic of the row
+        for (int i = tid; i < kSamples; i += kThreads) {
+            const int r = i / kSampleRun, j = i % kSampleRun;
+            const int64_t start = ((int64_t)r * n / (kSamples / kSampleRun)) & ~(int64_t)(kSampleRun - 1);
+            sm.key[i] = f32_order_key(row[min(start + j, (int64_t)n - 1)]);
+        }
         __syncthreads();
         const int64_t target = min((int64_t)2 * K, (int64_t)(K + kCap) / 2);
         const int rank = min(kSamples, (int)((target * kSamples + n - 1) / n) + 16);
+        // the sample's leading 16 bits suffice: the guess only has to lie at or
+        // below the rank-th sample (within 1/128 of it for positive scores)
         int unused;
-        radix_select([&](int i) { return sm.key[i]; }, kSamples, rank, sm, &guess, &unused);
+        radix_select([&](int i) { return sm.key[i]; }, kSamples, rank, sm, &guess, &unused, 2);
     }
 
     // 2. one pass: ordered compaction of the scores at or above the guess.  Each
