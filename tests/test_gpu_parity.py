@@ -285,6 +285,42 @@ def test_sparse_attn_parity(csa, H, K, win_count):
         assert attn_rel_err(o[b], ref) <= ATTN_REL
 
 
+@pytest.mark.parametrize("H,K,win_count,qexp", [(64, 512, 130, 17), (16, 100, 5, 17), (64, 256, 40, -20)])
+def test_sparse_attn_query_magnitude(csa, H, K, win_count, qexp):
+    """Queries 2^qexp times larger (|q| near 1e5, beyond fp16's range) or smaller
+    (near fp16's subnormals) with the scale 2^-qexp times smaller: the same
+    softmax, so the same output within the usual tolerance."""
+    B, T = 2, 2 * K + 50
+    wl = W.small(W.WORKLOADS[0], B=B, T=T, H=H, K=K)
+    dc = _dev_cache_from_recipe(csa, wl, 0, T)
+    rc = ref_cache(wl, 0, range(B), T, cap=T // 2 + 64)
+    n = T // 2
+    rng = np.random.default_rng(K + 1)
+    idx = np.stack([np.sort(rng.choice(n, size=K, replace=False)) for _ in range(B)]).astype(np.int32)
+    win = csa.engine.DeviceWindow(B, DEV)
+    rings = []
+    for b in range(B):
+        ring, _ = ref_window(wl, 0, b, win_count)
+        rings.append(ring)
+        win.tokens[b] = bf16_dev(ring)
+    win.count.fill_(win_count)
+    q0 = np.asarray(W.query(wl, 0, 0), np.uint16)
+    f = (q0.astype(np.uint32) << 16).view(np.float32) * np.float32(2.0 ** qexp)
+    q = (f.view(np.uint32) >> 16).astype(np.uint16)  # exact: a power-of-two multiple of bf16 values
+    assert np.array_equal((q.astype(np.uint32) << 16).view(np.float32), f)
+    scale = float(np.float32(wl.scale) * np.float32(2.0 ** -qexp))
+    out = torch.empty(B, H, 512, dtype=torch.float32, device=DEV)
+    ws = torch.empty(csa.sparse_attn_workspace(B, H, K), dtype=torch.uint8, device=DEV)
+    csa.sparse_attn(dc.desc, bf16_dev(q), torch.from_numpy(idx).to(DEV), K, win.desc, scale, out, ws)
+    torch.cuda.synchronize()
+    o = out.cpu().numpy()
+    assert np.isfinite(o).all()
+    for b in range(B):
+        items = oracle.attention_items(rc.mc[b], rc.ms[b], n, idx[b], rings[b], min(win_count, 128))
+        ref = oracle.attention(q[b], items, scale)
+        assert attn_rel_err(o[b], ref) <= ATTN_REL
+
+
 def test_window_append_ring(csa):
     B = 3
     win = csa.engine.DeviceWindow(B, DEV)
