@@ -4,15 +4,15 @@
 // Per (problem, sequence) the items are the K selected entries (dequantised
 // from E2M1 x E4M3: exact in fp16) and the valid window tokens (bf16 -> fp16,
 // exact for |x| in fp16's normal range, saturated at +-65504; E4M3 -> fp16,
-// always exact, for an FP8 window); the latent item is key and value.  Each
-// head's bf16 query row is multiplied by a power of two 2^k_h that brings its
-// largest magnitude into [2^14, 2^15) before it is rounded to fp16 (exact for
-// every bf16 value within 2^24 of the row's maximum), and 2^-k_h is folded
-// into that head's softmax scale, so no query magnitude overflows.
+// always exact, for an FP8 window); the latent item is key and value.  The
+// unit's bf16 query is multiplied by a power of two 2^k that brings its largest
+// magnitude into [2^14, 2^15) before it is rounded to fp16 (exact for every
+// bf16 value within 2^28 of that maximum), and 2^-k is folded into the softmax
+// scale, so no query magnitude overflows.
 // Items go through 128-item tiles with an online softmax:
 //
 //   S^T[128 items x 64 heads] = Items . Q^T            (M = 128, N = 64, K = 512)
-//   P^T = exp(scale_h * S^T - m_h)                     (fp16, per item lane)
+//   P^T = exp(scale 2^-k S^T - m_h)                    (fp16, per item lane)
 //   O^T[4 x 128 latent x 64 heads] += Items^T . P^T    (M = 128, N = 64, K = 128)
 //
 // One shared-memory image of the tile serves both MMAs: 128-byte-swizzled
@@ -32,12 +32,15 @@
 //               row, or window slot) two tiles ahead, and prefetches the window
 //               rows and the next unit's query into L2;
 //   warps 2-5   softmax: thread = item row (TMEM lane), all 64 heads; P^T into
-//               shared memory, the per-lane partial row sums in TMEM; at the end
+//               shared memory; the per-lane partial row sums and a per-lane
+//               copy of the 64 reference maxima live in TMEM, so a tile's
+//               softmax reads no shared memory but its item's kind; at the end
 //               of a unit the O^T readout, normalised (or the split's partial);
-//   warps 6-13  gather: warp g owns slab g (latent channels 64g .. 64g + 63);
-//               each tile's entry bytes are loaded into registers a tile ahead
-//               and dequantised into the slab once the previous tile's O block
-//               that reads it has completed; bf16 window rows arrive by TMA
+//   warps 6-13  gather: warp g owns slab pair g / 2 (an O block) for half the
+//               rows; each tile's entry bytes are loaded into registers a tile
+//               ahead, four lanes to an entry's piece (whole lines per load),
+//               and dequantised into the slabs once the previous tile's O block
+//               that reads them has completed; bf16 window rows arrive by TMA
 //               (issued by warp 13, which waits for the last O block) and are
 //               converted in place; the unit's query is converted in the slab
 //               layout.
@@ -71,6 +74,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;      // O^T: 4 blocks x 64 heads
 constexpr uint32_t kColS = 256;    // S^T: 64 heads
 constexpr uint32_t kColL = 320;    // per-lane partial row sums of P: 64 heads
+constexpr uint32_t kColM = 384;    // per-lane copy of the reference maxima: 64 heads
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kGap2 = 8.0f * kLog2e;  // the reference maximum moves beyond e^8 (log2 units)
@@ -87,8 +91,8 @@ struct __align__(1024) Smem {
     int64_t src_row[2][kT];        // per tile buffer: entry row in the pools, or window row
     int kind[2][kT];               // 0 empty, 1 cache entry, 2 bf16 window token, 3 E4M3 window token
     int tile_win[2];               // the tile holds bf16 window rows (loaded by TMA)
-    float a2[2][kHp];              // per unit parity: scale * 2^-k_h * log2(e)
-    uint32_t qmax[kGathWarps][kHp];  // per slab: largest |q| bf16 magnitude bits of a head
+    float a2[2];                   // per unit parity: scale * 2^-k * log2(e)
+    uint32_t qmax[kGathWarps];     // per slab: largest |q| bf16 magnitude bits
     float mu2[kHp];                // reference maximum per head (log2 units)
     float alpha[kHp];              // O / row-sum rescale factor of a move
     float red[4][kHp];             // per-quadrant partial max / sum
@@ -286,7 +290,9 @@ __device__ void role_mma(Smem& sm, const AttnBatch& ab, int splits, int tps, uin
                 alive = wait_bar_warp(sm, &sm.it_full[c], it & 1u) && alive;
                 tc_fence_after();
                 if (alive) {
-#pragma unroll
+                    // rolled: unrolled, the compiler hoists all 64 descriptors of a
+                    // tile into registers the other warps need
+#pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk) {  // 16 latent channels per MMA
                         const int ks = 8 * c + kk;
                         const uint32_t off = (uint32_t)((ks >> 2) * (kT * 128) + (ks & 3) * 32) >> 4;
@@ -305,7 +311,7 @@ __device__ void role_mma(Smem& sm, const AttnBatch& ab, int splits, int tps, uin
             if (alive) {
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
-#pragma unroll
+#pragma unroll 1
                     for (int i = 0; i < 8; ++i) {  // 16 items per MMA
                         const uint32_t offa = (uint32_t)(2 * c * (kT * 128) + 2048 * i) >> 4;
                         const uint32_t offp = (uint32_t)(2048 * i) >> 4;
@@ -323,55 +329,57 @@ __device__ void role_mma(Smem& sm, const AttnBatch& ab, int splits, int tps, uin
 // ---------------------------------------------------------------- warps 6-13: gather
 
 // The unit's query, slab g (channels 64g .. 64g + 63) of all 64 head rows,
-// scaled per head by 2^k_h and rounded to fp16; lane l owns heads l and l + 32.
-// k_h brings the head's largest bf16 magnitude into [2^14, 2^15).
+// scaled by 2^k and rounded to fp16.  Eight lanes cover a head row's 128 bytes
+// of the slab (lane: chunk l & 7 of heads 4i + l / 8), so a load instruction
+// reads four whole lines.  k brings the query's largest bf16 magnitude into
+// [2^14, 2^15): a first pass finds it, a second (from L1 / L2) converts.
 __device__ void convert_query(Smem& sm, const AttnBatch& ab, const Unit& u, int g, uint32_t ku, bool alive) {
     const int lane = threadIdx.x & 31;
     const int H = ab.H;
-    const uint16_t* qb = ab.p[u.prob].q + (int64_t)u.b * H * D + 64 * g;
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-        const int h = lane + 32 * half;
-        uint4 w[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            w[c] = h < H ? __ldg(reinterpret_cast<const uint4*>(qb + (int64_t)h * D) + c) : make_uint4(0, 0, 0, 0);
-        uint32_t m = 0;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            m = __vmaxu2(m, w[c].x & 0x7FFF7FFFu);
-            m = __vmaxu2(m, w[c].y & 0x7FFF7FFFu);
-            m = __vmaxu2(m, w[c].z & 0x7FFF7FFFu);
-            m = __vmaxu2(m, w[c].w & 0x7FFF7FFFu);
+    const int c = lane & 7, h0 = lane >> 3;
+    const uint4* qb = reinterpret_cast<const uint4*>(ab.p[u.prob].q + (int64_t)u.b * H * D + 64 * g) + c;
+    uint32_t m = 0;
+#pragma unroll 4
+    for (int i = 0; i < kHp / 4; ++i) {
+        const int h = 4 * i + h0;
+        if (h < H) {
+            const uint4 w = __ldg(qb + (int64_t)h * (D / 8));
+            m = __vmaxu2(m, w.x & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w.y & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w.z & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w.w & 0x7FFF7FFFu);
         }
-        sm.qmax[g][h] = max(m & 0xFFFFu, m >> 16);
-        named_bar(kBarGath, 32 * kGathWarps);
-        uint32_t mh = 0;
-#pragma unroll
-        for (int j = 0; j < kGathWarps; ++j) mh = max(mh, sm.qmax[j][h]);
-        // bf16 magnitude bits: exponent field E = mh >> 7; the maximum lies in
-        // [2^(E-127), 2^(E-126)), so k = 141 - E puts it in [2^14, 2^15)
-        const int E = (int)(mh >> 7);
-        const int kx = mh == 0 ? 0 : min(126, 141 - E);
-        const float mul = __uint_as_float((uint32_t)(127 + kx) << 23);
-        if (g == 0) sm.a2[ku & 1][h] = ab.scale * __uint_as_float((uint32_t)(127 - kx) << 23) * kLog2e;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint32_t ws[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
-            uint4 o;
-            uint32_t* os = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const __half2 hv = __floats2half2_rn(__uint_as_float(ws[e] << 16) * mul,
-                                                     __uint_as_float(ws[e] & 0xFFFF0000u) * mul);
-                os[e] = *reinterpret_cast<const uint32_t*>(&hv);
-            }
-            if (alive) *reinterpret_cast<uint4*>(sm.q[g] + sw128(h, c)) = o;
-        }
-        // no barrier after the reads: the two halves use disjoint heads, and a
-        // warp writes this half's heads again (next unit) only after every warp
-        // has passed the other half's barrier
     }
+    m = __reduce_max_sync(0xffffffffu, max(m & 0xFFFFu, m >> 16));
+    if (lane == 0) sm.qmax[g] = m;
+    named_bar(kBarGath, 32 * kGathWarps);
+    uint32_t mq = 0;
+#pragma unroll
+    for (int j = 0; j < kGathWarps; ++j) mq = max(mq, sm.qmax[j]);
+    // bf16 magnitude bits: exponent field E = mq >> 7; the maximum lies in
+    // [2^(E-127), 2^(E-126)), so k = 141 - E puts it in [2^14, 2^15)
+    const int E = (int)(mq >> 7);
+    const int kx = mq == 0 ? 0 : min(126, 141 - E);
+    const float mul = __uint_as_float((uint32_t)(127 + kx) << 23);
+    if (g == 0 && lane == 0) sm.a2[ku & 1] = ab.scale * __uint_as_float((uint32_t)(127 - kx) << 23) * kLog2e;
+#pragma unroll 4
+    for (int i = 0; i < kHp / 4; ++i) {
+        const int h = 4 * i + h0;
+        const uint4 w = h < H ? __ldg(qb + (int64_t)h * (D / 8)) : make_uint4(0, 0, 0, 0);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        uint4 o;
+        uint32_t* os = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __half2 hv = __floats2half2_rn(__uint_as_float(ws[e] << 16) * mul,
+                                                 __uint_as_float(ws[e] & 0xFFFF0000u) * mul);
+            os[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        if (alive) *reinterpret_cast<uint4*>(sm.q[g] + sw128(h, c)) = o;
+    }
+    // qmax is written again at the next unit, after its q_empty wait: that needs
+    // every S^T of this unit, so every gather warp's writes of every tile of
+    // this unit, all made after its reads above
 }
 
 // bf16 pair -> f16x2, saturated to fp16's finite range
@@ -382,10 +390,22 @@ __device__ __forceinline__ uint32_t bf16x2_to_h2_sat(uint32_t w) {
     return *reinterpret_cast<const uint32_t*>(&hv);
 }
 
+// Gather warp g writes slab pair cp = g / 2 (channels 128 cp .. 128 cp + 127)
+// of rows 64 (g % 2) .. 64 (g % 2) + 63.  Lane l takes quarter q = l % 4 of the
+// pair (32 channels: slab 2 cp + q / 2, chunks 4 (q % 2) .. + 3) of rows
+// 64 (g % 2) + 8 j + l / 4, j < 8: four lanes read an entry's 64 code bytes of
+// the pair, so a load instruction reads eight entries' pieces, one line each.
+// The lanes of a store instruction start at rotated chunks (lanes of the odd
+// slab two chunks on), so every eight lanes hit distinct banks.
 __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps, int splits, int tps) {
     const int lane = threadIdx.x & 31;
-    const int g = (threadIdx.x >> 5) - kWarpGath;  // slab
-    uint8_t* slab = sm.items[g];
+    const int g = (threadIdx.x >> 5) - kWarpGath;
+    const int cp = g >> 1;                 // slab pair (O block)
+    const int q = lane & 3;                // quarter of the pair
+    const int rbase = 64 * (g & 1) + (lane >> 2);
+    uint8_t* slab = sm.items[2 * cp + (q >> 1)];
+    const int cb = 4 * (q & 1);            // first chunk of the quarter in its slab
+    const int rot = 2 * (q >> 1);          // chunk rotation of the odd slab
     bool alive = true;
     uint32_t it = 0, ku = 0, wn = 0, w_issued = 0;
     Unit u;
@@ -394,42 +414,44 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps,
         const AttnProblem& P = ab.p[u.prob];
         for (int t = u.t0; t < u.t1; ++t, ++it) {
             const int buf = it & 1;
-            alive = wait_bar_warp(sm, &sm.lk_full[buf], (it >> 1) & 1u) && alive;
-            // this tile's rows lane + 32 i: their kind, and the entry bytes of slab g
-            int kd[4];
-            uint4 c0[4], c1[4];
-            uint32_t sc[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = lane + 32 * i;
-                kd[i] = sm.kind[buf][r];
-                if (kd[i] == 1) {
-                    const int64_t rw = sm.src_row[buf][r];
-                    const uint4* cs = reinterpret_cast<const uint4*>(P.cache.main_codes + rw * MCB + 32 * g);
-                    c0[i] = __ldg(cs);
-                    c1[i] = __ldg(cs + 1);
-                    sc[i] = __ldg(reinterpret_cast<const uint32_t*>(P.cache.main_scales + rw * MSB + 4 * g));
-                } else {
-                    c0[i] = c1[i] = make_uint4(0, 0, 0, 0);
-                    sc[i] = 0;
-                }
-            }
-            const bool win = sm.tile_win[buf] != 0;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.lk_empty[buf]);
-
             if (t == u.t0) {
-                // the unit's query: once the previous unit's S^T MMAs have completed
+                // the unit's query, once the previous unit's S^T MMAs have completed
+                // (before this tile's entry loads, so their registers are not live
+                // across the conversion)
                 if (ku > 0) alive = wait_bar_warp(sm, &sm.q_empty, (ku - 1) & 1u) && alive;
                 convert_query(sm, ab, u, g, ku, alive);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.q_ready[ku & 1]);
             }
-            // slab g is free once the previous tile's O block g / 2 has completed
+            alive = wait_bar_warp(sm, &sm.lk_full[buf], (it >> 1) & 1u) && alive;
+            // this tile's rows: their kinds (2 bits each), and the entry bytes of
+            // this quarter (code words, and the two scale bytes, paired per register)
+            uint32_t kinds = 0;
+            uint4 cw[8];
+            uint32_t sc[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = rbase + 8 * j;
+                const int kj = sm.kind[buf][r];
+                kinds |= (uint32_t)kj << (2 * j);
+                if (kj == 1) {
+                    const int64_t rw = sm.src_row[buf][r];
+                    cw[j] = __ldg(reinterpret_cast<const uint4*>(P.cache.main_codes + rw * MCB + 64 * cp + 16 * q));
+                    sc[j >> 1] |= (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(P.cache.main_scales + rw * MSB +
+                                                                                    8 * cp + 2 * q))
+                                  << (16 * (j & 1));
+                } else {
+                    cw[j] = make_uint4(0, 0, 0, 0);
+                }
+            }
+            const bool win = sm.tile_win[buf] != 0;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.lk_empty[buf]);
+            // slab pair cp is free once the previous tile's O block cp has completed
             // (every gather warp waits for every tile in order, so the parity
             // never aliases an older phase)
-            if (it > 0) alive = wait_bar_warp(sm, &sm.o_blk[g >> 1], (it - 1) & 1u) && alive;
+            if (it > 0) alive = wait_bar_warp(sm, &sm.o_blk[cp], (it - 1) & 1u) && alive;
             if (win) {
                 // bf16 window rows by TMA, one 64-channel box per slab, covering all
                 // 128 rows of every slab: issued by the warp that waited for block 3
@@ -448,64 +470,62 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps,
             }
             if (alive) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = lane + 32 * i;
-                    if (kd[i] == 1) {
-                        const uint32_t cw[8] = {c0[i].x, c0[i].y, c0[i].z, c0[i].w, c1[i].x, c1[i].y, c1[i].z, c1[i].w};
+                for (int j = 0; j < 8; ++j) {
+                    const int r = rbase + 8 * j;
+                    const uint32_t kj = (kinds >> (2 * j)) & 3u;
+                    if (kj == 1) {
+                        // E2M1 codes x E4M3 scale (one per 16 channels) -> fp16, exact
+                        const uint32_t w4[4] = {cw[j].x, cw[j].y, cw[j].z, cw[j].w};
+                        const uint32_t scj = sc[j >> 1] >> (16 * (j & 1));
+                        const __half2 s2[2] = {__float2half2_rn(e4m3_decode_pos(scj & 0xFFu)),
+                                               __float2half2_rn(e4m3_decode_pos((scj >> 8) & 0xFFu))};
 #pragma unroll
-                        for (int c2 = 0; c2 < 4; ++c2) {  // chunks 2 c2, 2 c2 + 1 share scale byte c2
-                            const __half2 s2 = __float2half2_rn(e4m3_decode_pos((sc[i] >> (8 * c2)) & 0xFFu));
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const int w = (kk + rot) & 3;  // chunk cb + w: channels 8 w .. of the quarter
+                            uint4 o;
+                            uint32_t* os = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-                            for (int cc = 0; cc < 2; ++cc) {
-                                const int c = 2 * c2 + cc;
-                                uint4 o;
-                                uint32_t* os = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const uint32_t hh = e2m1x2_to_h2((cw[c] >> (8 * e)) & 0xFFu);
-                                    const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&hh), s2);
-                                    os[e] = *reinterpret_cast<const uint32_t*>(&v);
-                                }
-                                *reinterpret_cast<uint4*>(slab + sw128(r, c)) = o;
+                            for (int e = 0; e < 4; ++e) {
+                                const uint32_t hh = e2m1x2_to_h2((w4[w] >> (8 * e)) & 0xFFu);
+                                const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&hh), s2[w >> 1]);
+                                os[e] = *reinterpret_cast<const uint32_t*>(&v);
                             }
+                            *reinterpret_cast<uint4*>(slab + sw128(r, cb + w)) = o;
                         }
-                    } else if (kd[i] == 2) {
+                    } else if (kj == 2) {
                         // bf16 window row, landed by TMA in the slab layout: to fp16 in place
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            uint4* ptr = reinterpret_cast<uint4*>(slab + sw128(r, c));
+                        for (int kk = 0; kk < 4; ++kk) {
+                            uint4* ptr = reinterpret_cast<uint4*>(slab + sw128(r, cb + ((kk + rot) & 3)));
                             const uint4 x = *ptr;
                             *ptr = make_uint4(bf16x2_to_h2_sat(x.x), bf16x2_to_h2_sat(x.y), bf16x2_to_h2_sat(x.z),
                                               bf16x2_to_h2_sat(x.w));
                         }
-                    } else if (kd[i] == 3) {
-                        // E4M3 window row (slot t * 128 + r - K of the ring): the slab's 64 codes -> fp16 (exact)
+                    } else if (kj == 3) {
+                        // E4M3 window row (slot t * 128 + r - K of the ring): 32 codes -> fp16 (exact)
                         const int64_t rw = (int64_t)u.b * WIN + (t * kT + r - P.K);
-                        const uint4* src =
-                            reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(P.win) + rw * D + 64 * g);
+                        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(P.win) + rw * D +
+                                                                          128 * cp + 32 * q);
+                        const uint4 x0 = __ldg(src), x1 = __ldg(src + 1);
+                        const uint32_t wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const uint4 x = __ldg(src + q4);
-                            const uint32_t cw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                            for (int cc = 0; cc < 2; ++cc) {
-                                uint4 o;
-                                o.x = e4m3x2_to_h2(cw[2 * cc] & 0xFFFFu);
-                                o.y = e4m3x2_to_h2(cw[2 * cc] >> 16);
-                                o.z = e4m3x2_to_h2(cw[2 * cc + 1] & 0xFFFFu);
-                                o.w = e4m3x2_to_h2(cw[2 * cc + 1] >> 16);
-                                *reinterpret_cast<uint4*>(slab + sw128(r, 2 * q4 + cc)) = o;
-                            }
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const int w = (kk + rot) & 3;  // chunk cb + w: code bytes 8 w .. 8 w + 7
+                            const uint4 o = make_uint4(e4m3x2_to_h2(wv[2 * w] & 0xFFFFu), e4m3x2_to_h2(wv[2 * w] >> 16),
+                                                       e4m3x2_to_h2(wv[2 * w + 1] & 0xFFFFu),
+                                                       e4m3x2_to_h2(wv[2 * w + 1] >> 16));
+                            *reinterpret_cast<uint4*>(slab + sw128(r, cb + w)) = o;
                         }
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(slab + sw128(r, c)) = make_uint4(0, 0, 0, 0);
+                        for (int kk = 0; kk < 4; ++kk)
+                            *reinterpret_cast<uint4*>(slab + sw128(r, cb + ((kk + rot) & 3))) = make_uint4(0, 0, 0, 0);
                     }
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.it_full[g >> 1]);
+            if (lane == 0) mbar_arrive(&sm.it_full[cp]);
         }
         ++ku;
     }
@@ -558,9 +578,16 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, int splits, int tps,
             continue;
         }
         if (st < kHp) sm.mu2[st] = -INFINITY;
+        {
+            float v[32];
+#pragma unroll
+            for (int h = 0; h < 32; ++h) v[h] = -INFINITY;
+            tmem_st_32x32b_x32(tl + kColM, v);
+            tmem_st_32x32b_x32(tl + kColM + 32, v);
+        }
         alive = wait_bar_warp(sm, &sm.q_ready[ku & 1], (ku >> 1) & 1u) && alive;
         named_bar(kBarSoft, 32 * kSoftWarps);
-        const float* a2 = sm.a2[ku & 1];
+        const float a2 = sm.a2[ku & 1];
         for (int t = u.t0; t < u.t1; ++t, ++it) {
             const int buf = it & 1;
             alive = wait_bar_warp(sm, &sm.lk_full[buf], (it >> 1) & 1u) && alive;
@@ -569,31 +596,29 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, int splits, int tps,
             if (lane == 0) mbar_arrive(&sm.lk_empty[buf]);
             alive = wait_bar_warp(sm, &sm.s_full, it & 1u) && alive;
             tc_fence_after();
-            float y0[32], y1[32];
-            // log2-domain exponent of every head against its reference maximum
-            auto load_y = [&]() {
-                tmem_ld_32x32b_x32(tl + kColS, y0);
-                tmem_ld_32x32b_x32(tl + kColS + 32, y1);
+            // pass 1: does this item move a head's maximum?  (S^T and the lane's
+            // copy of the maxima from TMEM, a half at a time)
+            bool need = false;
+#pragma unroll 1  // unrolled, both halves' loads are hoisted together: 128 registers
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[32], mv[32];
+                tmem_ld_x32_nowait(tl + kColS + 32 * half, sv);
+                tmem_ld_x32_nowait(tl + kColM + 32 * half, mv);
+                tmem_wait_ld2(sv, mv);
 #pragma unroll
-                for (int h = 0; h < 32; ++h) {
-                    y0[h] = y0[h] * a2[h] - sm.mu2[h];
-                    y1[h] = y1[h] * a2[32 + h] - sm.mu2[32 + h];
-                }
-            };
-            load_y();
-            bool need = false;  // does this item move a head's maximum?
-#pragma unroll
-            for (int h = 0; h < 32; ++h) need |= (y0[h] > kGap2) | (y1[h] > kGap2);
+                for (int h = 0; h < 32; ++h)
+                    need |= fmaf(__uint_as_float(sv[h]), a2, -__uint_as_float(mv[h])) > kGap2;
+            }
             if (named_bar_or(kBarSoft, 32 * kSoftWarps, (ok && need) || !alive)) {
-                // rare: the tile's maximum per head over the valid items (S^T reloaded)
-                tmem_ld_32x32b_x32(tl + kColS, y0);
+                // rare: the tile's maximum per head over the valid items
 #pragma unroll
-                for (int h = 0; h < 32; ++h) y0[h] = ok ? y0[h] * a2[h] : -INFINITY;
-                sm.red[quad][lane] = warp_reduce_scatter32<true>(y0);
-                tmem_ld_32x32b_x32(tl + kColS + 32, y1);
+                for (int half = 0; half < 2; ++half) {
+                    float z[32];
+                    tmem_ld_32x32b_x32(tl + kColS + 32 * half, z);
 #pragma unroll
-                for (int h = 0; h < 32; ++h) y1[h] = ok ? y1[h] * a2[32 + h] : -INFINITY;
-                sm.red[quad][32 + lane] = warp_reduce_scatter32<true>(y1);
+                    for (int h = 0; h < 32; ++h) z[h] = ok ? z[h] * a2 : -INFINITY;
+                    sm.red[quad][32 * half + lane] = warp_reduce_scatter32<true>(z);
+                }
                 named_bar(kBarSoft, 32 * kSoftWarps);
                 bool resc = false;
                 if (st < kHp) {
@@ -622,26 +647,38 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, int splits, int tps,
                         tmem_st_32x32b_x32(tl + col, o);
                     }
                 }
-                load_y();  // against the updated maxima
+                // this lane's TMEM copy of the updated maxima
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) v[h] = sm.mu2[32 * half + h];
+                    tmem_st_32x32b_x32(tl + kColM + 32 * half, v);
+                }
             }
             // P^T is free once the previous tile's O has completed
             if (it > 0) alive = wait_bar_warp(sm, &sm.o_blk[3], (it - 1) & 1u) && alive;
-            store_p(sm.p, row, 0, ok, y0);
-            store_p(sm.p, row, 4, ok, y1);
-            // this lane's running row sums (of the rounded p) in TMEM
-            if (t == u.t0) {
-                tmem_st_32x32b_x32(tl + kColL, y0);
-                tmem_st_32x32b_x32(tl + kColL + 32, y1);
-            } else {
-                float l[32];
-                tmem_ld_32x32b_x32(tl + kColL, l);
+            // pass 2: p = exp2(scale 2^-k s - m) into P^T (fp16), and the lane's
+            // running row sums of the rounded p in TMEM
 #pragma unroll
-                for (int h = 0; h < 32; ++h) l[h] += y0[h];
-                tmem_st_32x32b_x32(tl + kColL, l);
-                tmem_ld_32x32b_x32(tl + kColL + 32, l);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[32], mv[32];
+                tmem_ld_x32_nowait(tl + kColS + 32 * half, sv);
+                tmem_ld_x32_nowait(tl + kColM + 32 * half, mv);
+                tmem_wait_ld2(sv, mv);
+                float y[32];
 #pragma unroll
-                for (int h = 0; h < 32; ++h) l[h] += y1[h];
-                tmem_st_32x32b_x32(tl + kColL + 32, l);
+                for (int h = 0; h < 32; ++h) y[h] = fmaf(__uint_as_float(sv[h]), a2, -__uint_as_float(mv[h]));
+                store_p(sm.p, row, 4 * half, ok, y);
+                if (t == u.t0) {
+                    tmem_st_32x32b_x32(tl + kColL + 32 * half, y);
+                } else {
+                    float l[32];
+                    tmem_ld_32x32b_x32(tl + kColL + 32 * half, l);
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) l[h] += y[h];
+                    tmem_st_32x32b_x32(tl + kColL + 32 * half, l);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -668,17 +705,19 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, int splits, int tps,
         if (alive) {
             float* dst = partial ? ab.part_o + (int64_t)u.unit * H * D : ab.p[u.prob].out + (int64_t)u.b * H * D;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                const int lat = 128 * c + row;  // O^T block c, lane = latent channel
+            for (int h0 = 0; h0 < H; h0 += 16) {
+                float lf[16];  // the normalisers of these 16 heads, in registers
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float o[32];
-                    tmem_ld_32x32b_x32(tl + kColO + 64 * c + 32 * half, o);
+                for (int h = 0; h < 16; ++h) lf[h] = partial ? 1.0f : sm.lfin[h0 + h];
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    const int lat = 128 * c + row;  // O^T block c, lane = latent channel
+                    float o[16];
+                    tmem_ld_32x32b_x16(tl + kColO + 64 * c + h0, o);
+                    float* d = dst + (int64_t)h0 * D + lat;
 #pragma unroll
-                    for (int h = 0; h < 32; ++h) {
-                        const int hd = 32 * half + h;
-                        if (hd < H) dst[(int64_t)hd * D + lat] = partial ? o[h] : o[h] * sm.lfin[hd];
-                    }
+                    for (int h = 0; h < 16; ++h)
+                        if (h0 + h < H) d[(int64_t)h * D] = o[h] * lf[h];
                 }
             }
             if (partial && st < H) {
