@@ -176,6 +176,15 @@ def sparse_attn(cache, q, idx, K: int, win: csa2_window, scale: float, out, ws, 
         "csa2_sparse_attn")
 
 
+def selftest_wait_timeout(status, timeout_us: int, stream=None):
+    """Make one bounded device wait run out (see csa2_selftest_wait_timeout):
+    CSA2_DEVERR_TIMEOUT is ORed into status[0] after timeout_us microseconds."""
+    f = lib().csa2_selftest_wait_timeout
+    f.restype = ctypes.c_int
+    f.argtypes = [_vp, ctypes.c_uint, _vp]
+    _ok(f(_ptr(status), int(timeout_us), _stream(stream)), "csa2_selftest_wait_timeout")
+
+
 def window_append(win: csa2_window, tok, stream=None):
     _ok(lib().csa2_window_append(ctypes.byref(win), _ptr(tok), _stream(stream)), "csa2_window_append")
 

@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 using namespace csa2;
 
@@ -79,6 +80,27 @@ extern "C" {
 int csa2_version(void) { return (0 << 16) | 1; }
 
 int csa2_injected_faults(void) { return g_injected_faults.load(std::memory_order_relaxed); }
+
+namespace {
+
+// One thread waits on a barrier that no thread arrives at: the bounded wait
+// gives up after limit_ns and reports it, as every kernel's waits do.
+__global__ void k_selftest_wait_timeout(uint32_t* status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    csa2::sm100::mbar_init(&bar, 1);
+    csa2::sm100::fence_mbar_init();
+    if (!csa2::sm100::mbar_wait_ns(&bar, 0, limit_ns)) atomicOr(status, CSA2_DEVERR_TIMEOUT);
+}
+
+}  // namespace
+
+int csa2_selftest_wait_timeout(uint32_t* status, unsigned timeout_us, csa2_stream stream) {
+    if (!status || (reinterpret_cast<uintptr_t>(status) & 3u)) return CSA2_ERR_INVALID_ARG;
+    const uint64_t us = timeout_us < 1u ? 1u : (timeout_us > 2000000u ? 2000000u : timeout_us);
+    k_selftest_wait_timeout<<<1, 32, 0, (cudaStream_t)stream>>>(status, us * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
 
 const char* csa2_strerror(int status) {
     switch (status) {

@@ -83,6 +83,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// mbar_wait with the bound given in nanoseconds.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_sleep(bar, parity, 1000000u)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+
 // Warp-uniform wait: every lane polls, the result is the AND over the warp.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
     const bool ok = mbar_wait(bar, parity);

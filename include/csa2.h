@@ -168,6 +168,22 @@ int csa2_version(void);
  */
 int csa2_injected_faults(void);
 
+/*
+ * Self-test of the kernels' bounded waits (the pages have no counterpart).
+ * Every wait of every kernel of this library on an mbarrier (a copy landing, an
+ * MMA completing, another warp's hand-over) gives up after a time bound, ORs
+ * CSA2_DEVERR_TIMEOUT into a status word and lets the kernel return instead of
+ * hanging.  This entry point launches one small kernel that makes such a wait
+ * run out on purpose: it waits on a barrier nothing arrives at, with a bound of
+ * timeout_us microseconds (clamped to [1, 2,000,000]), then ORs
+ * CSA2_DEVERR_TIMEOUT into *status and returns; no memory but *status is
+ * touched and the context stays usable.
+ *   status   device pointer to one uint32 (4-byte aligned), caller-owned.
+ * Returns CSA2_ERR_INVALID_ARG for a NULL status, CSA2_ERR_CUDA if the launch
+ * fails; asynchronous on `stream` like every entry point.
+ */
+int csa2_selftest_wait_timeout(uint32_t* status, unsigned timeout_us, csa2_stream stream);
+
 /* Static string for a csa2_status value (never NULL). */
 const char* csa2_strerror(int status);
 

@@ -70,6 +70,11 @@ def test_argument_checks_fail_before_launch(capi):
                                 ctypes.c_void_p(16), None, 0, None) == -1
     assert capi.index_topk_workspace(2, 1024, 64, 512) > 2 * 1024 * 4
     assert capi.sparse_attn_workspace(2, 64, 512) > 0
+    # the bounded-wait self-test: a NULL or misaligned status word is refused
+    f = lib.csa2_selftest_wait_timeout
+    f.argtypes = [ctypes.c_void_p, ctypes.c_uint, ctypes.c_void_p]
+    assert f(None, 10, None) == -1
+    assert f(ctypes.c_void_p(18), 10, None) == -1
 
 
 def test_cache_io_argument_checks(capi):

@@ -84,14 +84,18 @@ def test_config2_full_size(engine):
     torch.cuda.synchronize()
     assert dm.status_bits() == 0
     T_now = wl.T + 2
-    b = 5
-    for s, layers in ((3, (20, 21, 22, 39)), (0, (2, 3, 4))):
-        rc = ref_cache(wl, s, [b], T_now, cap=T_now // 2 + 64)
-        assert dm.caches[s].n_entries[b].item() == rc.n[0] == T_now // 2
-        _check_cache(dm.caches[s], rc, b, int(rc.n[0]), ranges=[(0, 4096), (int(rc.n[0]) - 4096, int(rc.n[0]))])
-        for l in layers:
-            _check_layer(dm, wl, l, b, 1, rc, T_now)
-    _check_layer(dm, wl, 0, b, 1, None, T_now)  # window-only layer
+    # every source: its Full layer, a Reindex and a Reuse layer (source 3 also the
+    # last layer), for a middle and the last sequence of the batch
+    layers_of = {0: (2, 3, 4), 1: (8, 9, 10), 2: (14, 15, 16), 3: (20, 21, 22, 39)}
+    for b in (5, 15):
+        for s, layers in layers_of.items():
+            rc = ref_cache(wl, s, [b], T_now, cap=T_now // 2 + 64)
+            assert dm.caches[s].n_entries[b].item() == rc.n[0] == T_now // 2
+            _check_cache(dm.caches[s], rc, b, int(rc.n[0]),
+                         ranges=[(0, 4096), (int(rc.n[0]) - 4096, int(rc.n[0]))])
+            for l in layers:
+                _check_layer(dm, wl, l, b, 1, rc, T_now)
+        _check_layer(dm, wl, 0, b, 1, None, T_now)  # window-only layer
 
 
 def test_config3_full_size_outliers(engine):
