@@ -43,6 +43,8 @@ def parse():
                     help="a profiling case of workloads.PROFILE_WORKLOADS instead of --config")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-layer", action="store_true",
+                    help="skip the layer-by-layer timing of the indexer and attention")
     ap.add_argument("--profile-steps", type=int, default=5)
     ap.add_argument("--measure", choices=["step", "cache_io"], default="step",
                     help="cache_io: prefix-cache export/import throughput of one source's sequences")
@@ -550,7 +552,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return
     # the same indexer + attention work layer by layer (no grouping of scans)
-    pl_ms, pl_calls = per_layer_path(dm, wl, stream) if world == 1 else (None, None)
+    pl_ms, pl_calls = per_layer_path(dm, wl, stream) if world == 1 and not args.no_per_layer else (None, None)
 
     L = wl.table.n_layers
     value = replicas.job_rate(L, world, ms / 1e3)
