@@ -10,6 +10,8 @@
 // warp takes one head at a time: scores (lane = item), softmax statistics by
 // warp shuffles, output accumulation (lane = 16 channels).  Partials
 // (max, sum, unnormalised output) are merged by k_attn_combine.
+#include <cstdlib>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -220,8 +222,17 @@ bool attn_mma_supported(const AttnBatch& ab);
 size_t attn_mma_workspace_bytes(int n_problems, int batch, int H, int Kmax);
 cudaError_t launch_attn_mma(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev);
 
+// CSA2_ATTN_CUDA_CORE=1 in the environment selects the CUDA-core attention for
+// every head count (to compare the two kernels; the tensor-core one is the
+// default for 1 .. 64 heads).  Read at every call, by the workspace query and
+// the launch alike.
+static bool attn_cuda_core_forced() {
+    const char* e = std::getenv("CSA2_ATTN_CUDA_CORE");
+    return e && e[0] == '1' && e[1] == 0;
+}
+
 size_t attn_workspace_bytes(int n_problems, int batch, int H, int Kmax) {
-    if (H >= 1 && H <= 64) return attn_mma_workspace_bytes(n_problems, batch, H, Kmax);
+    if (H >= 1 && H <= 64 && !attn_cuda_core_forced()) return attn_mma_workspace_bytes(n_problems, batch, H, Kmax);
     const size_t units = (size_t)n_problems * batch * n_splits(Kmax) * H;
     return units * D * sizeof(float) + units * 2 * sizeof(float);
 }
@@ -249,14 +260,14 @@ cudaError_t launch_attn_cuda(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* 
 }  // namespace
 
 cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t* ev) {
-    if (attn_mma_supported(ab)) return launch_attn_mma(ab, st, ev);
+    if (attn_mma_supported(ab) && !attn_cuda_core_forced()) return launch_attn_mma(ab, st, ev);
     return launch_attn_cuda(ab, st, ev);
 }
 
 int attn_mma_splits(int n_problems, int batch, int Kmax);
 
 int sparse_attn_launches(const AttnBatch& ab) {
-    if (attn_mma_supported(ab)) return attn_mma_splits(ab.n, ab.batch, ab.Kmax) > 1 ? 2 : 1;
+    if (attn_mma_supported(ab) && !attn_cuda_core_forced()) return attn_mma_splits(ab.n, ab.batch, ab.Kmax) > 1 ? 2 : 1;
     return 2;
 }
 

@@ -300,6 +300,12 @@ size_t csa2_sparse_attn_workspace(int batch, int H, int K);
  *   q     bf16 [batch][H][512];  idx int32 [batch][K] (may be NULL when K = 0);
  *   out   fp32 [batch][H][512].
  * H in 1..128, K in 0..2048.  `cache` may be NULL when K = 0.
+ * Kernels: 1..64 heads run on the tensor cores (fp16 operands: the query is
+ * scaled by a power of two per (sequence, layer) before its fp16 rounding, so
+ * any bf16 query is exact within 2^28 of its largest magnitude; bf16 window
+ * values beyond +-65504 saturate there); other head counts, or every head count
+ * when the environment variable CSA2_ATTN_CUDA_CORE is "1" at the call (and at
+ * the workspace query), run on the CUDA cores with bf16 kept exact.
  */
 int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int H, const int32_t* idx, int K,
                      const csa2_window* win, float scale, float* out, void* ws, size_t ws_bytes,

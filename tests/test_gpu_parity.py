@@ -321,6 +321,13 @@ def test_sparse_attn_query_magnitude(csa, H, K, win_count, qexp):
         assert attn_rel_err(o[b], ref) <= ATTN_REL
 
 
+def test_sparse_attn_cuda_core_selected_at_64_heads(csa, monkeypatch):
+    """CSA2_ATTN_CUDA_CORE=1 runs the CUDA-core kernel at 64 heads (the tensor-core
+    one's comparison point): same parity bar, workspace sized for it."""
+    monkeypatch.setenv("CSA2_ATTN_CUDA_CORE", "1")
+    test_sparse_attn_parity(csa, 64, 512, 130)
+
+
 def test_window_append_ring(csa):
     B = 3
     win = csa.engine.DeviceWindow(B, DEV)
