@@ -24,15 +24,15 @@
 // costs ~300-450 cycles even with an empty epilogue.  Two alternating
 // epilogue groups keep the loads of one pass off the critical path of the next.
 //
-// Persistent, warp-specialised CTA (576 threads, one CTA per SM):
-//   warp 0  producer: decodes the CTA's work items (the only warp that reads the
-//           item tables among the kernel parameters) into a descriptor in shared
-//           memory per query buffer; per item the query tiles, query scales and
-//           head weights of every problem of the subset (double-buffered), per
-//           tile the key codes by TMA (one 64-entry page per box, 64-byte
-//           swizzle) and their E8M0 scales by bulk copy into an 8-stage ring.
-//           Keys stream with an L2 evict-first policy.  Tile copies are issued by
-//           one lane with warp-uniform operands.
+// Persistent, warp-specialised CTA (608 threads, one CTA per SM):
+//   warps 0, 18  producers: warp 0 decodes the CTA's work items into a
+//           descriptor in shared memory per query buffer and loads per item the
+//           query tiles, query scales and head weights of every problem of the
+//           subset (double-buffered); both load the key tiles, alternately, into
+//           an 8-stage ring: the key codes by TMA (one 64-entry page per box,
+//           64-byte swizzle) and their E8M0 scales by bulk copy.  Keys stream
+//           with an L2 evict-first policy.  Tile copies are issued by one lane
+//           with warp-uniform operands.
 //   warp 1  MMA issuer: rearranges each stage's and each item's E8M0 scales into
 //           the 32x128-bit layout tcgen05.cp reads and copies them into TMEM, then
 //           issues one MMA pass per problem pair into one of three TMEM
@@ -81,7 +81,8 @@ constexpr int kAcc = 3;           // TMEM accumulators: pass p lands in p % kAcc
 constexpr int kGroups = 2;        // epilogue groups: group g drains the passes p with p % 2 == g
 constexpr int kEpiWarps = 8 * kGroups;  // per group one per (TMEM lane quadrant, problem of the pass)
 constexpr int kEpi0 = 2;          // first epilogue warp
-constexpr int kThreads = 32 * (kEpi0 + kEpiWarps);
+constexpr int kProd1 = kEpi0 + kEpiWarps;  // second producer warp: the odd tiles
+constexpr int kThreads = 32 * (kProd1 + 1);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = 0;                            // kAcc x 128 accumulator columns
 constexpr uint32_t kColSfa = 128 * kAcc;                   // kStages x 4 scale columns (keys)
@@ -129,7 +130,7 @@ struct __align__(1024) Smem {
     uint8_t sfb_tc[2][kMaxPasses][512];
     float w[2][kMaxSub][kHeads];
     ItemDesc desc[2];
-    int prow[kMaxChunk * 16];                // pool items: first physical key row of each slot
+    int prow[2][kMaxChunk * 16];             // pool items, per producer: first physical key row of each slot
     uint64_t full[kStages], empty[kStages];
     uint64_t qfull[2], qempty[2];
     uint64_t tfull[kAcc], tempty[kAcc];
@@ -248,12 +249,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tbase = __shfl_sync(0xffffffffu, sm.tmem_base, 0);
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0 || warp == kProd1) {
+        // ------------------------------------------------------------ producers
+        // Both warps walk the same items and number the CTA's tiles in order (g);
+        // producer pw loads the tiles with g % 2 == pw into stage g % kStages
+        // (kStages is even, so every use of a stage belongs to one producer).
+        // Producer 0 also decodes each item's descriptor and loads its queries:
+        // a tile of one problem costs one warp ~1,000 cycles of copy issue,
+        // more than the MMA warp's pass.
+        const uint32_t pw = warp == 0 ? 0u : 1u;
         const int batch = sb.p[0].cache.batch;
         const uint64_t pol_stream = policy_evict_first();
         const uint64_t pol_keep = policy_evict_last();
-        if (lane == 0) prefetch_tmap(&mp.queries);
+        if (lane == 0 && pw == 0) prefetch_tmap(&mp.queries);
         uint32_t g = 0, bslot = 0, bphase = 0;
         uint32_t issued = 0, issued_par = 0;  // per stage: a copy was issued, and its phase
         bool stop = false;
@@ -280,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // the query buffer (and its item descriptor) is free once the item two
             // back is done: its MMAs completed and every epilogue warp left it
+            if (pw == 0) {
             if (!mbar_wait_warp(&sm.qempty[bslot], bphase ^ 1)) {
                 if (lane == 0) raise_abort(sm, status);
                 break;
@@ -310,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             if (++bslot == 2) bslot = 0, bphase ^= 1;
+            }  // producer 0's descriptor and queries
             const CUtensorMap* kmap = pool ? &mp.keys8[src] : &mp.keys[src];
             if (pool) {
                 // physical first row of every pool block of the item (positions
@@ -339,11 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         else
                             atomicOr(status, CSA2_DEVERR_PAGE);
                     }
-                    sm.prow[i] = r;
+                    sm.prow[pw][i] = r;
                 }
                 __syncwarp();
             }
             for (int t = it.t0; t < it.t1; ++t, ++g) {
+                if ((g & 1u) != pw) continue;  // the other producer's tile
                 const uint32_t stage = g % kStages, sphase = (g / kStages) & 1u;
                 if (!mbar_wait_warp(&sm.empty[stage], sphase ^ 1)) {
                     if (lane == 0) raise_abort(sm, status);
@@ -351,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 if (pool) {
-                    const int prow = lane < 16 ? sm.prow[16 * (t - it.t0) + lane] : -1;
+                    const int prow = lane < 16 ? sm.prow[pw][16 * (t - it.t0) + lane] : -1;
                     const unsigned have = __ballot_sync(0xffffffffu, prow >= 0);
                     if (have == 0) {
                         mbar_arrive_w(&sm.full[stage]);
@@ -393,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             stop = stop || __any_sync(0xffffffffu, aborted(sm));
         }
         // the end of the CTA's work: a descriptor with no problems
-        if (!stop && mbar_wait_warp(&sm.qempty[bslot], bphase ^ 1)) {
+        if (pw == 0 && !stop && mbar_wait_warp(&sm.qempty[bslot], bphase ^ 1)) {
             if (lane == 0) {
                 sm.desc[bslot].nprob = 0;
                 mbar_arrive(&sm.qfull[bslot]);
