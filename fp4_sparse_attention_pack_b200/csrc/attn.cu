@@ -264,10 +264,10 @@ cudaError_t launch_sparse_attn(const AttnBatch& ab, cudaStream_t st, cudaEvent_t
     return launch_attn_cuda(ab, st, ev);
 }
 
-int attn_mma_splits(int n_problems, int batch, int Kmax);
+int attn_mma_launches(const AttnBatch& ab);
 
 int sparse_attn_launches(const AttnBatch& ab) {
-    if (attn_mma_supported(ab) && !attn_cuda_core_forced()) return attn_mma_splits(ab.n, ab.batch, ab.Kmax) > 1 ? 2 : 1;
+    if (attn_mma_supported(ab) && !attn_cuda_core_forced()) return attn_mma_launches(ab);
     return 2;
 }
 

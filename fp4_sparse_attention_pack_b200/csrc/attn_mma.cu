@@ -186,21 +186,71 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32]) {
     return v[0];
 }
 
-// The unit a CTA takes k-th (units are strided over the CTAs).
-struct Unit {
-    int unit, prob, b, t0, t1;
+constexpr int kMaxTail = 256;  // units left after the full rounds: fewer than the CTAs
+
+// Host-computed work plan (a kernel parameter): problems in decreasing order of
+// tile count; with one split, the units left after the full rounds over the
+// CTAs (r < n_tail): problem and sequence (prob << 16 | b) and first piece.
+struct AttnOrder {
+    int prob[kMaxProblems];
+    int n_tail;
+    int tail_pb[kMaxTail];
+    int tail_first[kMaxTail + 1];
 };
 
-__device__ __forceinline__ bool unit_at(const AttnBatch& ab, int splits, int tps, int k, Unit& u) {
-    const int unit = blockIdx.x + k * gridDim.x;
-    if (unit >= ab.n * ab.batch * splits) return false;
-    const int split = unit % splits, pb = unit / splits;
-    u.unit = unit;
-    u.b = pb % ab.batch;
-    u.prob = pb / ab.batch;
-    const int n_tiles = (ab.p[u.prob].K + WIN + kT - 1) / kT;
-    u.t0 = split * tps;
-    u.t1 = min(n_tiles, u.t0 + tps);
+__device__ __forceinline__ int tiles_of(const AttnBatch& ab, int prob) { return (ab.p[prob].K + WIN + kT - 1) / kT; }
+
+// The work item a CTA takes k-th: tiles [t0, t1) of (problem, sequence), the
+// whole output or a partial (O, m, l) in slot `unit` of the workspace.
+//  - splits > 1 (few units): unit = (problem, sequence, split), strided over
+//    the CTAs, every split a partial;
+//  - one split: whole units, problems in decreasing tile count, in full rounds
+//    of one unit per CTA; then the remaining units' tiles one by one (a unit
+//    of one tile whole, the tiles of a longer unit as partials, slot = the
+//    piece's number), so no CTA runs a whole unit more than the others.
+struct Unit {
+    int unit, prob, b, t0, t1;
+    bool partial;
+};
+
+__device__ __noinline__ bool unit_at(const AttnOrder& ord, const AttnBatch& ab, int splits, int tps, int k, Unit& u) {
+    if (splits > 1) {
+        const int unit = blockIdx.x + k * gridDim.x;
+        if (unit >= ab.n * ab.batch * splits) return false;
+        const int split = unit % splits, pb = unit / splits;
+        u.unit = unit;
+        u.b = pb % ab.batch;
+        u.prob = pb / ab.batch;
+        u.t0 = split * tps;
+        u.t1 = min(tiles_of(ab, u.prob), u.t0 + tps);
+        u.partial = true;
+        return true;
+    }
+    const int G = gridDim.x, units = ab.n * ab.batch, rounds = units / G;
+    if (k < rounds) {
+        const int v = blockIdx.x + k * G;
+        u.prob = ord.prob[v / ab.batch];
+        u.b = v % ab.batch;
+        u.t0 = 0;
+        u.t1 = tiles_of(ab, u.prob);
+        u.partial = false;
+        u.unit = -1;
+        return true;
+    }
+    const int piece = blockIdx.x + (k - rounds) * G;
+    if (piece >= ord.tail_first[ord.n_tail]) return false;
+    int lo = 0, hi = ord.n_tail - 1;  // the unit r with tail_first[r] <= piece < tail_first[r + 1]
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (ord.tail_first[mid] <= piece) lo = mid; else hi = mid - 1;
+    }
+    const int T = ord.tail_first[lo + 1] - ord.tail_first[lo];
+    u.prob = ord.tail_pb[lo] >> 16;
+    u.b = ord.tail_pb[lo] & 0xFFFF;
+    u.t0 = piece - ord.tail_first[lo];
+    u.t1 = u.t0 + 1;
+    u.partial = T > 1;
+    u.unit = piece;
     return true;
 }
 
@@ -212,15 +262,17 @@ __device__ __forceinline__ int window_len(const AttnProblem& P, int b) {
 
 // ---------------------------------------------------------------- warp 1: items and window
 
-__device__ void role_producer(Smem& sm, const AttnBatch& ab, int splits, int tps) {
+__device__ void role_producer(Smem& sm, const AttnBatch& ab, const AttnOrder& ord, int splits, int tps) {
     const int lane = threadIdx.x & 31;
     bool alive = true;
     uint32_t it = 0;
     Unit u;
-    for (int k = 0; unit_at(ab, splits, tps, k, u); ++k) {
+    if (lane == 0 && unit_at(ord, ab, splits, tps, 0, u) && u.t0 < u.t1)
+        bulk_prefetch_l2(ab.p[u.prob].q + (int64_t)u.b * ab.H * D, (uint32_t)(ab.H * D * 2));
+    for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
         // the next unit's query into L2 while this unit runs
         Unit nu;
-        if (lane == 0 && unit_at(ab, splits, tps, k + 1, nu) && nu.t0 < nu.t1)
+        if (lane == 0 && unit_at(ord, ab, splits, tps, k + 1, nu) && nu.t0 < nu.t1)
             bulk_prefetch_l2(ab.p[nu.prob].q + (int64_t)nu.b * ab.H * D, (uint32_t)(ab.H * D * 2));
         if (u.t0 >= u.t1) continue;
         const AttnProblem& P = ab.p[u.prob];
@@ -270,7 +322,7 @@ __device__ void role_producer(Smem& sm, const AttnBatch& ab, int splits, int tps
 
 // ---------------------------------------------------------------- warp 0: MMA issue
 
-__device__ void role_mma(Smem& sm, const AttnBatch& ab, int splits, int tps, uint32_t tbase) {
+__device__ void role_mma(Smem& sm, const AttnBatch& ab, const AttnOrder& ord, int splits, int tps, uint32_t tbase) {
     const uint32_t idesc_s = idesc_f16(128, kHp, 0, 0, 0);
     const uint32_t idesc_o = idesc_f16(128, kHp, 0, 1, 1);
     const uint64_t desc_items = smem_desc(sm.items[0], 16, 1024, kLayoutSw128);
@@ -280,7 +332,7 @@ __device__ void role_mma(Smem& sm, const AttnBatch& ab, int splits, int tps, uin
     bool alive = true;
     uint32_t it = 0, ku = 0;
     Unit u;
-    for (int k = 0; unit_at(ab, splits, tps, k, u); ++k) {
+    for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
         if (u.t0 >= u.t1) continue;
         alive = wait_bar_warp(sm, &sm.q_ready[ku & 1], (ku >> 1) & 1u) && alive;
         for (int t = u.t0; t < u.t1; ++t, ++it) {
@@ -397,7 +449,8 @@ __device__ __forceinline__ uint32_t bf16x2_to_h2_sat(uint32_t w) {
 // the pair, so a load instruction reads eight entries' pieces, one line each.
 // The lanes of a store instruction start at rotated chunks (lanes of the odd
 // slab two chunks on), so every eight lanes hit distinct banks.
-__device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps, int splits, int tps) {
+__device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps, const AttnOrder& ord, int splits,
+                            int tps) {
     const int lane = threadIdx.x & 31;
     const int g = (threadIdx.x >> 5) - kWarpGath;
     const int cp = g >> 1;                 // slab pair (O block)
@@ -409,7 +462,7 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps,
     bool alive = true;
     uint32_t it = 0, ku = 0, wn = 0, w_issued = 0;
     Unit u;
-    for (int k = 0; unit_at(ab, splits, tps, k, u); ++k) {
+    for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
         if (u.t0 >= u.t1) continue;
         const AttnProblem& P = ab.p[u.prob];
         for (int t = u.t0; t < u.t1; ++t, ++it) {
@@ -558,18 +611,19 @@ __device__ __forceinline__ void store_p(uint8_t* prow_base, int row, int c0, boo
     }
 }
 
-__device__ void role_softmax(Smem& sm, const AttnBatch& ab, int splits, int tps, uint32_t tbase) {
+__device__ void role_softmax(Smem& sm, const AttnBatch& ab, const AttnOrder& ord, int splits, int tps,
+                             uint32_t tbase) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int row = 32 * quad + lane;          // item row (S^T) / latent row (O^T) of this thread
     const int st = threadIdx.x - 32 * kWarpSoft;  // 0 .. 127: per-head work for st < 64
     const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
     const int H = ab.H;
-    const bool partial = splits > 1;
     bool alive = true;
     uint32_t it = 0, ku = 0;
     Unit u;
-    for (int k = 0; unit_at(ab, splits, tps, k, u); ++k) {
+    for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
+        const bool partial = u.partial;
         if (u.t0 >= u.t1) {  // a split without tiles: an empty partial
             if (partial && st < H) {
                 ab.part_ml[((int64_t)u.unit * H + st) * 2 + 0] = -INFINITY;
@@ -735,7 +789,8 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, int splits, int tps,
 // ---------------------------------------------------------------- kernel
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k_attn_mma(const __grid_constant__ AttnBatch ab, const __grid_constant__ AttnMaps maps, int splits, int tps) {
+    k_attn_mma(const __grid_constant__ AttnBatch ab, const __grid_constant__ AttnMaps maps,
+               const __grid_constant__ AttnOrder ord, int splits, int tps) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -760,9 +815,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpProd) {
         for (int i = lane; i < ab.n; i += 32)
             if (!ab.p[i].win_fp8) prefetch_tmap(&maps.win[i]);
-        Unit u0;
-        if (lane == 0 && unit_at(ab, splits, tps, 0, u0) && u0.t0 < u0.t1)
-            bulk_prefetch_l2(ab.p[u0.prob].q + (int64_t)u0.b * ab.H * D, (uint32_t)(ab.H * D * 2));
     }
     if (warp == kWarpMma) tmem_alloc(&sm.tmem_base, kTmemCols);
     tc_fence_before();
@@ -772,18 +824,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tbase = __shfl_sync(0xffffffffu, sm.tmem_base, 0);
 
     if (warp == kWarpMma)
-        role_mma(sm, ab, splits, tps, tbase);
+        role_mma(sm, ab, ord, splits, tps, tbase);
     else if (warp == kWarpProd)
-        role_producer(sm, ab, splits, tps);
+        role_producer(sm, ab, ord, splits, tps);
     else if (warp < kWarpGath)
-        role_softmax(sm, ab, splits, tps, tbase);
+        role_softmax(sm, ab, ord, splits, tps, tbase);
     else
-        role_gather(sm, ab, maps, splits, tps);
+        role_gather(sm, ab, maps, ord, splits, tps);
 
     __syncthreads();
     if (sm.abort && tid == 0) {  // report on the first of this CTA's units that has a cache
         Unit u;
-        for (int k = 0; unit_at(ab, splits, tps, k, u); ++k)
+        for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k)
             if (ab.p[u.prob].K > 0) {
                 atomicOr(ab.p[u.prob].cache.status, CSA2_DEVERR_TIMEOUT);
                 break;
@@ -802,32 +854,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// out = sum_s O_s e^(m_s - M) / sum_s l_s e^(m_s - M) over the splits of (problem, sequence)
-__global__ void k_attn_mma_combine(const __grid_constant__ AttnBatch ab, int splits) {
-    const int h = blockIdx.x, b = blockIdx.y, prob = blockIdx.z;
-    const AttnProblem& P = ab.p[prob];
+// out[j] = sum_s O_s[j] e^(m_s - M) / sum_s l_s e^(m_s - M) over the partials in
+// slots slot0 .. slot0 + n - 1 of head h (threadIdx.x: channels x, x + 128, ...).
+__device__ void merge_partials(const AttnBatch& ab, int64_t slot0, int n, int h, float* o) {
     const int H = ab.H;
-    const int64_t u0 = ((int64_t)prob * ab.batch + b) * splits;
     float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, ab.part_ml[((u0 + s) * H + h) * 2]);
+    for (int s = 0; s < n; ++s) M = fmaxf(M, ab.part_ml[((slot0 + s) * H + h) * 2]);
     float L = 0.0f;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (M != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
-            const float m = ab.part_ml[((u0 + s) * H + h) * 2];
-            const float l = ab.part_ml[((u0 + s) * H + h) * 2 + 1];
+        for (int s = 0; s < n; ++s) {
+            const float m = ab.part_ml[((slot0 + s) * H + h) * 2];
+            const float l = ab.part_ml[((slot0 + s) * H + h) * 2 + 1];
             if (m == -INFINITY || l == 0.0f) continue;
             const float f = expf(m - M);
             L += l * f;
-            const float* po = ab.part_o + ((u0 + s) * H + h) * D;
+            const float* po = ab.part_o + ((slot0 + s) * H + h) * D;
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[i] = fmaf(f, po[threadIdx.x + 128 * i], acc[i]);
         }
     }
-    float* o = P.out + ((int64_t)b * H + h) * D;
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[threadIdx.x + 128 * i] = acc[i] * inv;
+}
+
+// Every split of (problem, sequence) is a partial: merge them.
+__global__ void k_attn_mma_combine(const __grid_constant__ AttnBatch ab, int splits) {
+    const int h = blockIdx.x, b = blockIdx.y, prob = blockIdx.z;
+    merge_partials(ab, ((int64_t)prob * ab.batch + b) * splits, splits, h,
+                   ab.p[prob].out + ((int64_t)b * ab.H + h) * D);
+}
+
+// One split: the units after the full rounds ran tile by tile; merge the
+// pieces of each such unit longer than one tile (blockIdx.y: the r-th of them).
+__global__ void k_attn_mma_combine_tail(const __grid_constant__ AttnBatch ab, const __grid_constant__ AttnOrder ord,
+                                        int G) {
+    (void)G;
+    const int h = blockIdx.x, r = blockIdx.y;
+    const int p0 = ord.tail_first[r], T = ord.tail_first[r + 1] - p0;
+    if (T == 1) return;  // written whole by its CTA
+    const int prob = ord.tail_pb[r] >> 16, b = ord.tail_pb[r] & 0xFFFF;
+    merge_partials(ab, p0, T, h, ab.p[prob].out + ((int64_t)b * ab.H + h) * D);
 }
 
 }  // namespace
@@ -843,11 +911,64 @@ int attn_mma_splits(int n_problems, int batch, int Kmax) {
 
 bool attn_mma_supported(const AttnBatch& ab) { return ab.H >= 1 && ab.H <= kHp; }
 
-size_t attn_mma_workspace_bytes(int n_problems, int batch, int H, int Kmax) {
+// CTAs of a launch over `units` work units: one per SM, at most one per unit
+// (and at most kMaxTail, the size of the plan's tail table).
+static int attn_grid(int units) { return std::min(std::min(units, device_sm_count()), kMaxTail); }
+
+// Partial slots of a launch: every split, or (one split) at most every tile of
+// the units left after the full rounds over the CTAs.
+static size_t attn_mma_slots(int n_problems, int batch, int Kmax) {
     const int splits = attn_mma_splits(n_problems, batch, Kmax);
-    if (splits == 1) return 0;
-    const size_t units = (size_t)n_problems * batch * splits;
-    return units * H * D * sizeof(float) + units * H * 2 * sizeof(float);
+    const int units = n_problems * batch;
+    if (splits > 1) return (size_t)units * splits;
+    const int G = attn_grid(units);
+    const int rem = G > 0 ? units % G : 0;
+    return (size_t)rem * ((Kmax + WIN + kT - 1) / kT);
+}
+
+size_t attn_mma_workspace_bytes(int n_problems, int batch, int H, int Kmax) {
+    const size_t slots = attn_mma_slots(n_problems, batch, Kmax);
+    return slots * H * D * sizeof(float) + slots * H * 2 * sizeof(float);
+}
+
+namespace {
+
+// The work plan of a launch on G CTAs: problems in decreasing tile count (ties
+// in problem order) and, with one split, the units left after the full rounds.
+AttnOrder attn_order(const AttnBatch& ab, int splits, int G) {
+    AttnOrder o;
+    std::memset(&o, 0, sizeof(o));
+    for (int i = 0; i < ab.n; ++i) o.prob[i] = i;
+    std::stable_sort(o.prob, o.prob + ab.n, [&](int a, int b) { return ab.p[a].K > ab.p[b].K; });
+    if (splits == 1 && G > 0) {
+        const int units = ab.n * ab.batch, rounds = units / G;
+        int first = 0;
+        for (int v = rounds * G; v < units; ++v) {
+            const int r = o.n_tail++;
+            const int prob = o.prob[v / ab.batch];
+            o.tail_pb[r] = prob << 16 | (v % ab.batch);
+            o.tail_first[r] = first;
+            first += (ab.p[prob].K + WIN + kT - 1) / kT;
+        }
+        o.tail_first[o.n_tail] = first;
+    }
+    return o;
+}
+
+// Does a unit of the tail have more than one tile (so the tail merge runs)?
+bool attn_tail_merge(const AttnOrder& o) {
+    for (int r = 0; r < o.n_tail; ++r)
+        if (o.tail_first[r + 1] - o.tail_first[r] > 1) return true;
+    return false;
+}
+
+}  // namespace
+
+int attn_mma_launches(const AttnBatch& ab) {
+    const int splits = attn_mma_splits(ab.n, ab.batch, ab.Kmax);
+    if (splits > 1) return 2;
+    const int units = ab.n * ab.batch;
+    return 1 + (attn_tail_merge(attn_order(ab, 1, attn_grid(units))) ? 1 : 0);
 }
 
 namespace {
@@ -888,23 +1009,26 @@ cudaError_t launch_attn_mma(const AttnBatch& ab_in, cudaStream_t st, cudaEvent_t
     const int splits = attn_mma_splits(ab.n, ab.batch, ab.Kmax);
     const int tiles = (ab.Kmax + WIN + kT - 1) / kT;
     const int tps = (tiles + splits - 1) / splits;
-    if (splits > 1) {
-        const size_t units = (size_t)ab.n * ab.batch * splits;
-        ab.part_ml = ab.part_o + units * ab.H * D;
-    }
+    const size_t slots = attn_mma_slots(ab.n, ab.batch, ab.Kmax);
+    if (slots > 0) ab.part_ml = ab.part_o + slots * ab.H * D;
     const int units = ab.n * ab.batch * splits;
-    const int grid = std::min(units, device_sm_count());
+    const int grid = attn_grid(units);
+    const AttnOrder ord = attn_order(ab, splits, grid);
     const size_t smem = sizeof(Smem) + 1024;
     static std::atomic<uint64_t> attr_done{0};
     const cudaError_t ea = smem_opt_in(reinterpret_cast<const void*>(k_attn_mma), (int)smem, attr_done);
     if (ea != cudaSuccess) return ea;
-    k_attn_mma<<<grid, kThreads, smem, st>>>(ab, maps, splits, tps);
+    k_attn_mma<<<grid, kThreads, smem, st>>>(ab, maps, ord, splits, tps);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (ev) cudaEventRecord(ev[0], st);
     if (splits > 1) {
         dim3 g(ab.H, ab.batch, ab.n);
         k_attn_mma_combine<<<g, 128, 0, st>>>(ab, splits);
+        e = cudaGetLastError();
+    } else if (attn_tail_merge(ord)) {
+        dim3 g(ab.H, ord.n_tail);
+        k_attn_mma_combine_tail<<<g, 128, 0, st>>>(ab, ord, grid);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess && ev) cudaEventRecord(ev[1], st);

@@ -328,6 +328,35 @@ def test_sparse_attn_cuda_core_selected_at_64_heads(csa, monkeypatch):
     test_sparse_attn_parity(csa, 64, 512, 130)
 
 
+def test_sparse_attn_tail_tiles_merged(csa):
+    """More (sequence) units than SMs: after one unit per CTA, the remaining
+    units run tile by tile as partials merged by the tail kernel; every
+    sequence, those included, matches the oracle."""
+    B, T, K, H, wc = 150, 600, 256, 16, 40
+    wl = W.small(W.WORKLOADS[0], B=B, T=T, H=H, K=K)
+    dc = _dev_cache_from_recipe(csa, wl, 0, T)
+    rc = ref_cache(wl, 0, range(B), T, cap=T // 2 + 64)
+    n = T // 2
+    rng = np.random.default_rng(7)
+    idx = np.stack([np.sort(rng.choice(n, size=K, replace=False)) for _ in range(B)]).astype(np.int32)
+    win = csa.engine.DeviceWindow(B, DEV)
+    rings = []
+    for b in range(B):
+        ring, _ = ref_window(wl, 0, b, wc)
+        rings.append(ring)
+        win.tokens[b] = bf16_dev(ring)
+    win.count.fill_(wc)
+    q = W.query(wl, 0, 0)
+    out = torch.empty(B, H, 512, dtype=torch.float32, device=DEV)
+    ws = torch.empty(max(csa.sparse_attn_workspace(B, H, K), 16), dtype=torch.uint8, device=DEV)
+    csa.sparse_attn(dc.desc, bf16_dev(q), torch.from_numpy(idx).to(DEV), K, win.desc, wl.scale, out, ws)
+    torch.cuda.synchronize()
+    o = out.cpu().numpy()
+    for b in (0, 1, 146, 147, 148, 149):
+        items = oracle.attention_items(rc.mc[b], rc.ms[b], n, idx[b], rings[b], wc)
+        assert attn_rel_err(o[b], oracle.attention(q[b], items, wl.scale)) <= ATTN_REL, b
+
+
 def test_window_append_ring(csa):
     B = 3
     win = csa.engine.DeviceWindow(B, DEV)
