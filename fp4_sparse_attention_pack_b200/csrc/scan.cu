@@ -66,28 +66,38 @@ __global__ void k_quant_queries(ScanBatch sb, int batch) {
     const int g = blockIdx.x * blockDim.x + threadIdx.x;  // (b, h, blk)
     if (g >= batch * H * 4) return;
     const int blk = g & 3, bh = g >> 2;
-    const uint16_t* src = P.q_idx + (int64_t)bh * DI + 32 * blk;
+    // the block's 32 bf16 values: four 16-byte loads (rows are 256-byte aligned)
+    const uint4* src = reinterpret_cast<const uint4*>(P.q_idx + (int64_t)bh * DI + 32 * blk);
     const int64_t qrow = (int64_t)prob * batch * H + bh;  // row of (problem, sequence, head)
     float v[32];
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        v[i] = bf16_bits_to_f32(src[i]);
-        amax = fmaxf(amax, fabsf(v[i]));
-    }
-    uint8_t* dst = sb.qc + qrow * ICB + 16 * blk;
-    if (amax == 0.0f) {
+    for (int c = 0; c < 4; ++c) {
+        const uint4 w = __ldg(src + c);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dst[i] = 0;
+        for (int k = 0; k < 4; ++k) {
+            v[8 * c + 2 * k] = __uint_as_float(ws[k] << 16);
+            v[8 * c + 2 * k + 1] = __uint_as_float(ws[k] & 0xFFFF0000u);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    uint4* dst = reinterpret_cast<uint4*>(sb.qc + qrow * ICB + 16 * blk);
+    if (amax == 0.0f) {
+        *dst = make_uint4(0, 0, 0, 0);
         sb.qs[qrow * ISB + blk] = 0;
         return;
     }
     const int X = mx_shared_exp(amax);
     const float inv = pow2i(-X);
+    uint32_t cw[4] = {0, 0, 0, 0};  // 32 codes, channel 2i in the low nibble of byte i
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-        dst[i] = (uint8_t)(e2m1_encode(__fmul_rn(v[2 * i], inv)) |
-                           (e2m1_encode(__fmul_rn(v[2 * i + 1], inv)) << 4));
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t byte = e2m1_encode(__fmul_rn(v[2 * i], inv)) | (e2m1_encode(__fmul_rn(v[2 * i + 1], inv)) << 4);
+        cw[i >> 2] |= byte << (8 * (i & 3));
+    }
+    *dst = make_uint4(cw[0], cw[1], cw[2], cw[3]);
     sb.qs[qrow * ISB + blk] = (uint8_t)(X + 127);
 }
 
