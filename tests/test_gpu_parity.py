@@ -357,6 +357,43 @@ def test_sparse_attn_tail_tiles_merged(csa):
         assert attn_rel_err(o[b], oracle.attention(q[b], items, wl.scale)) <= ATTN_REL, b
 
 
+def test_sparse_attn_window_beyond_fp16_saturates(csa):
+    """Tensor-core attention: bf16 window values beyond fp16's range saturate at
+    +-65504 (the header's contract): outputs stay finite and equal the oracle's
+    on the clamped window."""
+    B, T, K, H, wc = 2, 600, 128, 64, 20
+    wl = W.small(W.WORKLOADS[0], B=B, T=T, H=H, K=K)
+    dc = _dev_cache_from_recipe(csa, wl, 0, T)
+    rc = ref_cache(wl, 0, range(B), T, cap=T // 2 + 64)
+    n = T // 2
+    rng = np.random.default_rng(11)
+    idx = np.stack([np.sort(rng.choice(n, size=K, replace=False)) for _ in range(B)]).astype(np.int32)
+    win = csa.engine.DeviceWindow(B, DEV)
+    rings, clamped = [], []
+    for b in range(B):
+        ring, _ = ref_window(wl, 0, b, wc)
+        f = (np.asarray(ring, np.uint16).astype(np.uint32) << 16).view(np.float32).copy()
+        f[3, :64] *= np.float32(2.0 ** 20)   # one token with channels near 1e5 .. 1e6
+        bits = (f.view(np.uint32) >> 16).astype(np.uint16)
+        rings.append(bits)
+        c = np.clip((bits.astype(np.uint32) << 16).view(np.float32), -65504.0, 65504.0)
+        clamped.append(c)
+        win.tokens[b] = bf16_dev(bits)
+    win.count.fill_(wc)
+    q = W.query(wl, 0, 0)
+    scale = float(np.float32(wl.scale) * np.float32(2.0 ** -12))  # keep the softmax away from one-hot
+    out = torch.empty(B, H, 512, dtype=torch.float32, device=DEV)
+    ws = torch.empty(max(csa.sparse_attn_workspace(B, H, K), 16), dtype=torch.uint8, device=DEV)
+    csa.sparse_attn(dc.desc, bf16_dev(q), torch.from_numpy(idx).to(DEV), K, win.desc, scale, out, ws)
+    torch.cuda.synchronize()
+    o = out.cpu().numpy()
+    assert np.isfinite(o).all()
+    for b in range(B):
+        items = oracle.attention_items(rc.mc[b], rc.ms[b], n, idx[b], rings[b], wc)
+        items[K:K + wc] = clamped[b][:wc]  # the window rows as the kernel reads them
+        assert attn_rel_err(o[b], oracle.attention(q[b], items, scale)) <= ATTN_REL
+
+
 def test_window_append_ring(csa):
     B = 3
     win = csa.engine.DeviceWindow(B, DEV)
