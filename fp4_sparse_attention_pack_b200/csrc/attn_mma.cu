@@ -100,8 +100,8 @@ struct __align__(1024) Smem {
     uint64_t lk_full[2], lk_empty[2];  // item lookups: producer -> gather + softmax warps
     uint64_t q_ready[2];           // the unit's query converted (per unit parity)
     uint64_t q_empty;              // every S^T MMA of the unit completed
-    uint64_t w_full;               // window TMA landed
-    uint64_t it_full[4];           // slab pair c of the tile written
+    uint64_t w_full[4];            // window TMA of slab pair c landed
+    uint64_t it_full[4];           // slab pair c of the tile written (every gather warp)
     uint64_t s_full;               // S^T complete
     uint64_t p_full;               // P^T written, S^T read
     uint64_t o_blk[4];             // O^T block c complete (block 3: the whole tile)
@@ -442,25 +442,23 @@ __device__ __forceinline__ uint32_t bf16x2_to_h2_sat(uint32_t w) {
     return *reinterpret_cast<const uint32_t*>(&hv);
 }
 
-// Gather warp g writes slab pair cp = g / 2 (channels 128 cp .. 128 cp + 127)
-// of rows 64 (g % 2) .. 64 (g % 2) + 63.  Lane l takes quarter q = l % 4 of the
-// pair (32 channels: slab 2 cp + q / 2, chunks 4 (q % 2) .. + 3) of rows
-// 64 (g % 2) + 8 j + l / 4, j < 8: four lanes read an entry's 64 code bytes of
-// the pair, so a load instruction reads eight entries' pieces, one line each.
-// The lanes of a store instruction start at rotated chunks (lanes of the odd
-// slab two chunks on), so every eight lanes hit distinct banks.
+// The eight gather warps write every slab pair of a tile together, pair after
+// pair, each as soon as the previous tile's O block that reads it has
+// completed, so a pair is ready a few hundred cycles after its block: thread
+// (g, l) owns half h = l % 2 of row 16 g + l / 2 of every pair c, i.e. slab
+// 2 c + h of that row (64 channels: 32 code bytes, four scale bytes, one
+// 128-byte line of the image).  Odd lanes store their chunks four on, so that
+// every eight lanes of a store hit distinct banks.  All of a tile's entry bytes
+// are loaded into registers before the first pair's wait.
 __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps, const AttnOrder& ord, int splits,
                             int tps) {
     const int lane = threadIdx.x & 31;
     const int g = (threadIdx.x >> 5) - kWarpGath;
-    const int cp = g >> 1;                 // slab pair (O block)
-    const int q = lane & 3;                // quarter of the pair
-    const int rbase = 64 * (g & 1) + (lane >> 2);
-    uint8_t* slab = sm.items[2 * cp + (q >> 1)];
-    const int cb = 4 * (q & 1);            // first chunk of the quarter in its slab
-    const int rot = 2 * (q >> 1);          // chunk rotation of the odd slab
+    const int r = 16 * g + (lane >> 1);  // item row
+    const int hf = lane & 1;             // slab 2 c + hf of pair c
     bool alive = true;
-    uint32_t it = 0, ku = 0, wn = 0, w_issued = 0;
+    uint32_t it = 0, ku = 0, wn = 0;
+    uint32_t wiss = 0, wpar = 0;  // bit c: a window copy of pair c was issued; parity of their count
     Unit u;
     for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
         if (u.t0 >= u.t1) continue;
@@ -478,112 +476,123 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps,
                 if (lane == 0) mbar_arrive(&sm.q_ready[ku & 1]);
             }
             alive = wait_bar_warp(sm, &sm.lk_full[buf], (it >> 1) & 1u) && alive;
-            // this tile's rows: their kinds (2 bits each), and the entry bytes of
-            // this quarter (code words, and the two scale bytes, paired per register)
-            uint32_t kinds = 0;
-            uint4 cw[8];
-            uint32_t sc[4] = {0, 0, 0, 0};
+            // this row's kind, and (an entry) its code words and scale bytes of
+            // every pair's half
+            const int kind = sm.kind[buf][r];
+            uint4 cw[4][2];
+            uint32_t sc[4];
+            if (kind == 1) {
+                const int64_t rw = sm.src_row[buf][r];
+                const uint8_t* codes = P.cache.main_codes + rw * MCB + 32 * hf;
+                const uint8_t* scl = P.cache.main_scales + rw * MSB + 4 * hf;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = rbase + 8 * j;
-                const int kj = sm.kind[buf][r];
-                kinds |= (uint32_t)kj << (2 * j);
-                if (kj == 1) {
-                    const int64_t rw = sm.src_row[buf][r];
-                    cw[j] = __ldg(reinterpret_cast<const uint4*>(P.cache.main_codes + rw * MCB + 64 * cp + 16 * q));
-                    sc[j >> 1] |= (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(P.cache.main_scales + rw * MSB +
-                                                                                    8 * cp + 2 * q))
-                                  << (16 * (j & 1));
-                } else {
-                    cw[j] = make_uint4(0, 0, 0, 0);
+                for (int c = 0; c < 4; ++c) {
+                    cw[c][0] = __ldg(reinterpret_cast<const uint4*>(codes + 64 * c));
+                    cw[c][1] = __ldg(reinterpret_cast<const uint4*>(codes + 64 * c + 16));
+                    sc[c] = __ldg(reinterpret_cast<const uint32_t*>(scl + 8 * c));
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    cw[c][0] = cw[c][1] = make_uint4(0, 0, 0, 0);
+                    sc[c] = 0;
                 }
             }
             const bool win = sm.tile_win[buf] != 0;
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.lk_empty[buf]);
-            // slab pair cp is free once the previous tile's O block cp has completed
-            // (every gather warp waits for every tile in order, so the parity
-            // never aliases an older phase)
-            if (it > 0) alive = wait_bar_warp(sm, &sm.o_blk[cp], (it - 1) & 1u) && alive;
-            if (win) {
-                // bf16 window rows by TMA, one 64-channel box per slab, covering all
-                // 128 rows of every slab: issued by the warp that waited for block 3
-                // (the previous tile's last O block, so all of its O)
-                if (g == kGathWarps - 1 && alive) {
-                    if (lane == 0) {
-                        mbar_expect_tx(&sm.w_full, 8 * kT * 128);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            tma_load_3d(sm.items[j], &maps.win[u.prob], 64 * j, t * kT - P.K, u.b, &sm.w_full);
+            for (int c = 0; c < 4; ++c) {
+                // pair c is free once the previous tile's O block c has completed
+                // (every gather warp waits for every block of every tile in order,
+                // so the parity never aliases an older phase)
+                if (it > 0) alive = wait_bar_warp(sm, &sm.o_blk[c], (it - 1) & 1u) && alive;
+                if (win) {
+                    // bf16 window rows of the pair by TMA (two 64-channel boxes over
+                    // all 128 rows), issued by gather warp 0; rows that are not
+                    // window tokens are rewritten below, after it lands
+                    if (g == 0 && alive) {
+                        if (lane == 0) {
+                            mbar_expect_tx(&sm.w_full[c], 2 * kT * 128);
+                            tma_load_3d(sm.items[2 * c], &maps.win[u.prob], 128 * c, t * kT - P.K, u.b, &sm.w_full[c]);
+                            tma_load_3d(sm.items[2 * c + 1], &maps.win[u.prob], 128 * c + 64, t * kT - P.K, u.b,
+                                        &sm.w_full[c]);
+                        }
+                        wiss |= 1u << c;
+                        wpar ^= 1u << c;
                     }
-                    ++w_issued;
+                    alive = wait_bar_warp(sm, &sm.w_full[c], wn & 1u) && alive;
                 }
-                alive = wait_bar_warp(sm, &sm.w_full, wn & 1u) && alive;
-                ++wn;
-            }
-            if (alive) {
+                uint8_t* line = sm.items[2 * c + hf];
+                if (alive) {
+                    if (kind == 1) {
+                        // E2M1 codes x E4M3 scale (one per 16 channels) -> fp16, exact:
+                        // chunk w holds channels 8 w .. 8 w + 7 (code word w, scale w / 2)
+                        const uint32_t w8[8] = {cw[c][0].x, cw[c][0].y, cw[c][0].z, cw[c][0].w,
+                                                cw[c][1].x, cw[c][1].y, cw[c][1].z, cw[c][1].w};
+                        __half2 s2[4];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r = rbase + 8 * j;
-                    const uint32_t kj = (kinds >> (2 * j)) & 3u;
-                    if (kj == 1) {
-                        // E2M1 codes x E4M3 scale (one per 16 channels) -> fp16, exact
-                        const uint32_t w4[4] = {cw[j].x, cw[j].y, cw[j].z, cw[j].w};
-                        const uint32_t scj = sc[j >> 1] >> (16 * (j & 1));
-                        const __half2 s2[2] = {__float2half2_rn(e4m3_decode_pos(scj & 0xFFu)),
-                                               __float2half2_rn(e4m3_decode_pos((scj >> 8) & 0xFFu))};
+                        for (int j = 0; j < 4; ++j) s2[j] = __float2half2_rn(e4m3_decode_pos((sc[c] >> (8 * j)) & 0xFFu));
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const int w = (kk + rot) & 3;  // chunk cb + w: channels 8 w .. of the quarter
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const int w0 = kk, w1 = (kk + 4) & 7;  // odd lanes: four chunks on
+                            const uint32_t word = hf ? w8[w1] : w8[w0];
+                            const __half2 s = hf ? s2[w1 >> 1] : s2[w0 >> 1];
                             uint4 o;
                             uint32_t* os = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const uint32_t hh = e2m1x2_to_h2((w4[w] >> (8 * e)) & 0xFFu);
-                                const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&hh), s2[w >> 1]);
+                                const uint32_t hh = e2m1x2_to_h2((word >> (8 * e)) & 0xFFu);
+                                const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&hh), s);
                                 os[e] = *reinterpret_cast<const uint32_t*>(&v);
                             }
-                            *reinterpret_cast<uint4*>(slab + sw128(r, cb + w)) = o;
+                            *reinterpret_cast<uint4*>(line + sw128(r, hf ? w1 : w0)) = o;
                         }
-                    } else if (kj == 2) {
+                    } else if (kind == 2) {
                         // bf16 window row, landed by TMA in the slab layout: to fp16 in place
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            uint4* ptr = reinterpret_cast<uint4*>(slab + sw128(r, cb + ((kk + rot) & 3)));
+                        for (int kk = 0; kk < 8; ++kk) {
+                            uint4* ptr = reinterpret_cast<uint4*>(line + sw128(r, hf ? ((kk + 4) & 7) : kk));
                             const uint4 x = *ptr;
                             *ptr = make_uint4(bf16x2_to_h2_sat(x.x), bf16x2_to_h2_sat(x.y), bf16x2_to_h2_sat(x.z),
                                               bf16x2_to_h2_sat(x.w));
                         }
-                    } else if (kj == 3) {
-                        // E4M3 window row (slot t * 128 + r - K of the ring): 32 codes -> fp16 (exact)
+                    } else if (kind == 3) {
+                        // E4M3 window row (slot t * 128 + r - K of the ring): 64 codes -> fp16 (exact)
                         const int64_t rw = (int64_t)u.b * WIN + (t * kT + r - P.K);
                         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(P.win) + rw * D +
-                                                                          128 * cp + 32 * q);
-                        const uint4 x0 = __ldg(src), x1 = __ldg(src + 1);
-                        const uint32_t wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                                                                          128 * c + 64 * hf);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const int w = (kk + rot) & 3;  // chunk cb + w: code bytes 8 w .. 8 w + 7
-                            const uint4 o = make_uint4(e4m3x2_to_h2(wv[2 * w] & 0xFFFFu), e4m3x2_to_h2(wv[2 * w] >> 16),
-                                                       e4m3x2_to_h2(wv[2 * w + 1] & 0xFFFFu),
-                                                       e4m3x2_to_h2(wv[2 * w + 1] >> 16));
-                            *reinterpret_cast<uint4*>(slab + sw128(r, cb + w)) = o;
+                        for (int q = 0; q < 4; ++q) {  // 16 codes: chunks 2 q, 2 q + 1
+                            const uint4 x = __ldg(src + (hf ? ((q + 2) & 3) : q));
+                            const int c0 = hf ? ((2 * q + 4) & 7) : 2 * q;
+                            *reinterpret_cast<uint4*>(line + sw128(r, c0)) =
+                                make_uint4(e4m3x2_to_h2(x.x & 0xFFFFu), e4m3x2_to_h2(x.x >> 16),
+                                           e4m3x2_to_h2(x.y & 0xFFFFu), e4m3x2_to_h2(x.y >> 16));
+                            *reinterpret_cast<uint4*>(line + sw128(r, c0 + 1)) =
+                                make_uint4(e4m3x2_to_h2(x.z & 0xFFFFu), e4m3x2_to_h2(x.z >> 16),
+                                           e4m3x2_to_h2(x.w & 0xFFFFu), e4m3x2_to_h2(x.w >> 16));
                         }
                     } else {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            *reinterpret_cast<uint4*>(slab + sw128(r, cb + ((kk + rot) & 3))) = make_uint4(0, 0, 0, 0);
+                        for (int kk = 0; kk < 8; ++kk)
+                            *reinterpret_cast<uint4*>(line + sw128(r, kk)) = make_uint4(0, 0, 0, 0);
                     }
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.it_full[c]);
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.it_full[cp]);
+            if (win) ++wn;
         }
         ++ku;
     }
-    // a window copy that was issued but not waited for lands before the CTA exits
-    if (!alive && w_issued > 0 && lane == 0) (void)mbar_wait(&sm.w_full, (w_issued - 1) & 1u);
+    // window copies that were issued but not waited for land before the CTA exits
+    if (!alive && g == 0 && lane == 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if ((wiss >> c) & 1u) (void)mbar_wait(&sm.w_full[c], ((wpar >> c) & 1u) ^ 1u);
+    }
 }
 
 // ---------------------------------------------------------------- warps 2-5: softmax
@@ -801,9 +810,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.q_ready[i], kGathWarps);
         }
         mbar_init(&sm.q_empty, 1);
-        mbar_init(&sm.w_full, 1);
+        for (int c = 0; c < 4; ++c) mbar_init(&sm.w_full[c], 1);
         for (int c = 0; c < 4; ++c) {
-            mbar_init(&sm.it_full[c], 2);
+            mbar_init(&sm.it_full[c], kGathWarps);
             mbar_init(&sm.o_blk[c], 1);
         }
         mbar_init(&sm.s_full, 1);
