@@ -23,7 +23,7 @@
 // cross-item reduction at all: every thread tests its own item against m_h and
 // one barrier ORs the tests.
 //
-// Persistent CTAs (one per SM, 448 threads) walk their units (problem,
+// Persistent CTAs (one per SM, 480 threads) walk their units (problem,
 // sequence, split of tiles) tile by tile; warps specialise and hand work over
 // through mbarriers, never through a block-wide barrier:
 //   warp 0      issues the MMAs (one elected lane): S^T of a tile slab pair by
@@ -36,14 +36,15 @@
 //               copy of the 64 reference maxima live in TMEM, so a tile's
 //               softmax reads no shared memory but its item's kind; at the end
 //               of a unit the O^T readout, normalised (or the split's partial);
-//   warps 6-13  gather: warp g owns slab pair g / 2 (an O block) for half the
-//               rows; each tile's entry bytes are loaded into registers a tile
-//               ahead, four lanes to an entry's piece (whole lines per load),
-//               and dequantised into the slabs once the previous tile's O block
-//               that reads them has completed; bf16 window rows arrive by TMA
-//               (issued by warp 13, which waits for the last O block) and are
-//               converted in place; the unit's query is converted in the slab
-//               layout.
+//   warps 6-13  gather: all eight write each slab pair of a tile (an O block's
+//               operand) together, pair after pair, as soon as the previous
+//               tile's O block that reads it has completed; each tile's entry
+//               bytes are loaded into registers before the first pair's wait;
+//               bf16 window rows are converted in place once their TMA lands;
+//               the unit's query is converted in the slab layout;
+//   warp 14     window: loads each tile's bf16 window rows by TMA, slab pair by
+//               slab pair as the O blocks complete, so a pair's copy is in
+//               flight while the gather converts the pair before it.
 // A waiter only ever waits for the phase right after the last one it saw
 // complete: a wait further ahead would alias an older phase of the same parity.
 #include <cuda.h>
@@ -69,7 +70,8 @@ constexpr int kT = 128;            // items per tile (MMA M of S^T)
 constexpr int kHp = 64;            // heads, padded (MMA N)
 constexpr int kWarpMma = 0, kWarpProd = 1, kWarpSoft = 2, kWarpGath = 6;
 constexpr int kSoftWarps = 4, kGathWarps = 8;
-constexpr int kThreads = 32 * (kWarpGath + kGathWarps);  // 448
+constexpr int kWarpWin = kWarpGath + kGathWarps;         // window TMA issuer
+constexpr int kThreads = 32 * (kWarpWin + 1);             // 480
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;      // O^T: 4 blocks x 64 heads
 constexpr uint32_t kColS = 256;    // S^T: 64 heads
@@ -450,15 +452,13 @@ __device__ __forceinline__ uint32_t bf16x2_to_h2_sat(uint32_t w) {
 // 128-byte line of the image).  Odd lanes store their chunks four on, so that
 // every eight lanes of a store hit distinct banks.  All of a tile's entry bytes
 // are loaded into registers before the first pair's wait.
-__device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps, const AttnOrder& ord, int splits,
-                            int tps) {
+__device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnOrder& ord, int splits, int tps) {
     const int lane = threadIdx.x & 31;
     const int g = (threadIdx.x >> 5) - kWarpGath;
     const int r = 16 * g + (lane >> 1);  // item row
     const int hf = lane & 1;             // slab 2 c + hf of pair c
     bool alive = true;
     uint32_t it = 0, ku = 0, wn = 0;
-    uint32_t wiss = 0, wpar = 0;  // bit c: a window copy of pair c was issued; parity of their count
     Unit u;
     for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
         if (u.t0 >= u.t1) continue;
@@ -507,22 +507,9 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps,
                 // (every gather warp waits for every block of every tile in order,
                 // so the parity never aliases an older phase)
                 if (it > 0) alive = wait_bar_warp(sm, &sm.o_blk[c], (it - 1) & 1u) && alive;
-                if (win) {
-                    // bf16 window rows of the pair by TMA (two 64-channel boxes over
-                    // all 128 rows), issued by gather warp 0; rows that are not
-                    // window tokens are rewritten below, after it lands
-                    if (g == 0 && alive) {
-                        if (lane == 0) {
-                            mbar_expect_tx(&sm.w_full[c], 2 * kT * 128);
-                            tma_load_3d(sm.items[2 * c], &maps.win[u.prob], 128 * c, t * kT - P.K, u.b, &sm.w_full[c]);
-                            tma_load_3d(sm.items[2 * c + 1], &maps.win[u.prob], 128 * c + 64, t * kT - P.K, u.b,
-                                        &sm.w_full[c]);
-                        }
-                        wiss |= 1u << c;
-                        wpar ^= 1u << c;
-                    }
-                    alive = wait_bar_warp(sm, &sm.w_full[c], wn & 1u) && alive;
-                }
+                // bf16 window rows of the pair arrive by TMA (the window warp's);
+                // rows that are not window tokens are rewritten below, after it lands
+                if (win) alive = wait_bar_warp(sm, &sm.w_full[c], wn & 1u) && alive;
                 uint8_t* line = sm.items[2 * c + hf];
                 if (alive) {
                     if (kind == 1) {
@@ -587,8 +574,46 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnMaps& maps,
         }
         ++ku;
     }
-    // window copies that were issued but not waited for land before the CTA exits
-    if (!alive && g == 0 && lane == 0) {
+}
+
+// The window warp: for every tile, in order, waits for the previous tile's O
+// block c and (a tile with bf16 window tokens) loads slab pair c of the window
+// rows by TMA: two 64-channel boxes over the tile's 128 rows, so the copy of a
+// pair is in flight while the gather warps convert the pair before it.
+__device__ void role_window(Smem& sm, const AttnBatch& ab, const AttnMaps& maps, const AttnOrder& ord, int splits,
+                            int tps) {
+    const int lane = threadIdx.x & 31;
+    bool alive = true;
+    uint32_t it = 0;
+    uint32_t wiss = 0, wpar = 0;  // bit c: a copy of pair c was issued; parity of their count
+    Unit u;
+    for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
+        if (u.t0 >= u.t1) continue;
+        const AttnProblem& P = ab.p[u.prob];
+        const int wlen = window_len(P, u.b);
+        for (int t = u.t0; t < u.t1; ++t, ++it) {
+            // the lookup warp's test for kind-2 rows: window slots t kT - K .. + kT - 1
+            // that are below the window length
+            const bool win = !P.win_fp8 && wlen > 0 && t * kT + kT > P.K && t * kT < P.K + wlen;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                // every block of every tile in order (the parity never aliases)
+                if (it > 0) alive = wait_bar_warp(sm, &sm.o_blk[c], (it - 1) & 1u) && alive;
+                if (win && alive) {
+                    if (lane == 0) {
+                        mbar_expect_tx(&sm.w_full[c], 2 * kT * 128);
+                        tma_load_3d(sm.items[2 * c], &maps.win[u.prob], 128 * c, t * kT - P.K, u.b, &sm.w_full[c]);
+                        tma_load_3d(sm.items[2 * c + 1], &maps.win[u.prob], 128 * c + 64, t * kT - P.K, u.b,
+                                    &sm.w_full[c]);
+                    }
+                    wiss |= 1u << c;
+                    wpar ^= 1u << c;
+                }
+            }
+        }
+    }
+    // copies that were issued but not waited for land before the CTA exits
+    if (!alive && lane == 0) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
             if ((wiss >> c) & 1u) (void)mbar_wait(&sm.w_full[c], ((wpar >> c) & 1u) ^ 1u);
@@ -838,8 +863,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         role_producer(sm, ab, ord, splits, tps);
     else if (warp < kWarpGath)
         role_softmax(sm, ab, ord, splits, tps, tbase);
+    else if (warp < kWarpWin)
+        role_gather(sm, ab, ord, splits, tps);
     else
-        role_gather(sm, ab, maps, ord, splits, tps);
+        role_window(sm, ab, maps, ord, splits, tps);
 
     __syncthreads();
     if (sm.abort && tid == 0) {  // report on the first of this CTA's units that has a cache
