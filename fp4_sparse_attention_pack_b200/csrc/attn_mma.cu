@@ -94,14 +94,14 @@ struct __align__(1024) Smem {
     int kind[2][kT];               // 0 empty, 1 cache entry, 2 bf16 window token, 3 E4M3 window token
     int tile_win[2];               // the tile holds bf16 window rows (loaded by TMA)
     float a2[2];                   // per unit parity: scale * 2^-k * log2(e)
-    uint32_t qmax[kGathWarps];     // per slab: largest |q| bf16 magnitude bits
+    uint32_t qmax[2][kGathWarps];  // per unit parity and slab: largest |q| bf16 magnitude bits
     float mu2[kHp];                // reference maximum per head (log2 units)
     float alpha[kHp];              // O / row-sum rescale factor of a move
     float red[4][kHp];             // per-quadrant partial max / sum
     float lfin[kHp];               // row sum of the unit
     uint64_t lk_full[2], lk_empty[2];  // item lookups: producer -> gather + softmax warps
-    uint64_t q_ready[2];           // the unit's query converted (per unit parity)
-    uint64_t q_empty;              // every S^T MMA of the unit completed
+    uint64_t q_ready[2][4];        // the unit's query slab pair c converted (per unit parity)
+    uint64_t q_empty[4];           // every S^T MMA of the unit that reads query slab pair c completed
     uint64_t w_full[4];            // window TMA of slab pair c landed
     uint64_t it_full[4];           // slab pair c of the tile written (every gather warp)
     uint64_t s_full;               // S^T complete
@@ -336,12 +336,14 @@ __device__ void role_mma(Smem& sm, const AttnBatch& ab, const AttnOrder& ord, in
     Unit u;
     for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
         if (u.t0 >= u.t1) continue;
-        alive = wait_bar_warp(sm, &sm.q_ready[ku & 1], (ku >> 1) & 1u) && alive;
         for (int t = u.t0; t < u.t1; ++t, ++it) {
             // S^T = Items . Q^T, slab pair by slab pair as the gather warps finish them
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 alive = wait_bar_warp(sm, &sm.it_full[c], it & 1u) && alive;
+                // the unit's query slab pair c (converted pair by pair as the previous
+                // unit's last S^T releases it)
+                if (t == u.t0) alive = wait_bar_warp(sm, &sm.q_ready[ku & 1][c], (ku >> 1) & 1u) && alive;
                 tc_fence_after();
                 if (alive) {
                     // rolled: unrolled, the compiler hoists all 64 descriptors of a
@@ -353,12 +355,11 @@ __device__ void role_mma(Smem& sm, const AttnBatch& ab, const AttnOrder& ord, in
                         const uint32_t offq = (uint32_t)((ks >> 2) * (kHp * 128) + (ks & 3) * 32) >> 4;
                         tc_mma_f16_w(tbase + kColS, desc_items + off, desc_q + offq, idesc_s, ks > 0 ? 1u : 0u);
                     }
+                    // the unit's last S^T frees query slab pair c for the next unit
+                    if (t + 1 == u.t1) tc_commit_w(&sm.q_empty[c]);
                 }
             }
-            if (alive) {
-                tc_commit_w(&sm.s_full);
-                if (t + 1 == u.t1) tc_commit_w(&sm.q_empty);
-            }
+            if (alive) tc_commit_w(&sm.s_full);
             // O^T += Items^T . P^T, one commit per 128-channel block (slabs 2c, 2c + 1)
             alive = wait_bar_warp(sm, &sm.p_full, it & 1u) && alive;
             tc_fence_after();
@@ -386,8 +387,11 @@ __device__ void role_mma(Smem& sm, const AttnBatch& ab, const AttnOrder& ord, in
 // scaled by 2^k and rounded to fp16.  Eight lanes cover a head row's 128 bytes
 // of the slab (lane: chunk l & 7 of heads 4i + l / 8), so a load instruction
 // reads four whole lines.  k brings the query's largest bf16 magnitude into
-// [2^14, 2^15): a first pass finds it, a second (from L1 / L2) converts.
-__device__ void convert_query(Smem& sm, const AttnBatch& ab, const Unit& u, int g, uint32_t ku, bool alive) {
+// [2^14, 2^15): a first pass finds it, a second (from L1 / L2) converts, once
+// the previous unit's last S^T has read the slab's pair (the first pass runs
+// before: the conversion of a unit's query overlaps the end of the previous
+// unit).
+__device__ bool convert_query(Smem& sm, const AttnBatch& ab, const Unit& u, int g, uint32_t ku, bool alive) {
     const int lane = threadIdx.x & 31;
     const int H = ab.H;
     const int c = lane & 7, h0 = lane >> 3;
@@ -405,17 +409,19 @@ __device__ void convert_query(Smem& sm, const AttnBatch& ab, const Unit& u, int 
         }
     }
     m = __reduce_max_sync(0xffffffffu, max(m & 0xFFFFu, m >> 16));
-    if (lane == 0) sm.qmax[g] = m;
+    if (lane == 0) sm.qmax[ku & 1][g] = m;
     named_bar(kBarGath, 32 * kGathWarps);
     uint32_t mq = 0;
 #pragma unroll
-    for (int j = 0; j < kGathWarps; ++j) mq = max(mq, sm.qmax[j]);
+    for (int j = 0; j < kGathWarps; ++j) mq = max(mq, sm.qmax[ku & 1][j]);
     // bf16 magnitude bits: exponent field E = mq >> 7; the maximum lies in
     // [2^(E-127), 2^(E-126)), so k = 141 - E puts it in [2^14, 2^15)
     const int E = (int)(mq >> 7);
     const int kx = mq == 0 ? 0 : min(126, 141 - E);
     const float mul = __uint_as_float((uint32_t)(127 + kx) << 23);
     if (g == 0 && lane == 0) sm.a2[ku & 1] = ab.scale * __uint_as_float((uint32_t)(127 - kx) << 23) * kLog2e;
+    // slab g is free once the previous unit's last S^T has read its pair
+    if (ku > 0) alive = wait_bar_warp(sm, &sm.q_empty[g >> 1], (ku - 1) & 1u) && alive;
 #pragma unroll 4
     for (int i = 0; i < kHp / 4; ++i) {
         const int h = 4 * i + h0;
@@ -431,17 +437,19 @@ __device__ void convert_query(Smem& sm, const AttnBatch& ab, const Unit& u, int 
         }
         if (alive) *reinterpret_cast<uint4*>(sm.q[g] + sw128(h, c)) = o;
     }
-    // qmax is written again at the next unit, after its q_empty wait: that needs
-    // every S^T of this unit, so every gather warp's writes of every tile of
-    // this unit, all made after its reads above
+    // qmax[ku & 1] is written again two units on, after every gather warp has
+    // passed the next unit's barrier, so after every read above
+    return alive;
 }
 
-// bf16 pair -> f16x2, saturated to fp16's finite range
+// bf16 pair -> f16x2 (round to nearest), saturated to fp16's finite range: one
+// conversion instruction whose .satfinite clamps a result beyond +-65504 to it
 __device__ __forceinline__ uint32_t bf16x2_to_h2_sat(uint32_t w) {
-    const float lo = fminf(fmaxf(__uint_as_float(w << 16), -65504.0f), 65504.0f);
-    const float hi = fminf(fmaxf(__uint_as_float(w & 0xFFFF0000u), -65504.0f), 65504.0f);
-    const __half2 hv = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&hv);
+    uint32_t d;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;"
+        : "=r"(d)
+        : "f"(__uint_as_float(w & 0xFFFF0000u)), "f"(__uint_as_float(w << 16)));  // (high, low)
+    return d;
 }
 
 // The eight gather warps write every slab pair of a tile together, pair after
@@ -466,14 +474,12 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnOrder& ord,
         for (int t = u.t0; t < u.t1; ++t, ++it) {
             const int buf = it & 1;
             if (t == u.t0) {
-                // the unit's query, once the previous unit's S^T MMAs have completed
-                // (before this tile's entry loads, so their registers are not live
-                // across the conversion)
-                if (ku > 0) alive = wait_bar_warp(sm, &sm.q_empty, (ku - 1) & 1u) && alive;
-                convert_query(sm, ab, u, g, ku, alive);
+                // the unit's query (before this tile's entry loads, so their
+                // registers are not live across the conversion)
+                alive = convert_query(sm, ab, u, g, ku, alive);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.q_ready[ku & 1]);
+                if (lane == 0) mbar_arrive(&sm.q_ready[ku & 1][g >> 1]);
             }
             alive = wait_bar_warp(sm, &sm.lk_full[buf], (it >> 1) & 1u) && alive;
             // this row's kind, and (an entry) its code words and scale bytes of
@@ -673,7 +679,9 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, const AttnOrder& ord
             tmem_st_32x32b_x32(tl + kColM, v);
             tmem_st_32x32b_x32(tl + kColM + 32, v);
         }
-        alive = wait_bar_warp(sm, &sm.q_ready[ku & 1], (ku >> 1) & 1u) && alive;
+        // the unit's scale (written by the gather warp of query slab 0 before its
+        // arrival on pair 0)
+        alive = wait_bar_warp(sm, &sm.q_ready[ku & 1][0], (ku >> 1) & 1u) && alive;
         named_bar(kBarSoft, 32 * kSoftWarps);
         const float a2 = sm.a2[ku & 1];
         for (int t = u.t0; t < u.t1; ++t, ++it) {
@@ -832,9 +840,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.lk_full[i], 1);
             mbar_init(&sm.lk_empty[i], kGathWarps + kSoftWarps);
-            mbar_init(&sm.q_ready[i], kGathWarps);
+            for (int c = 0; c < 4; ++c) mbar_init(&sm.q_ready[i][c], 2);
         }
-        mbar_init(&sm.q_empty, 1);
+        for (int c = 0; c < 4; ++c) mbar_init(&sm.q_empty[c], 1);
         for (int c = 0; c < 4; ++c) mbar_init(&sm.w_full[c], 1);
         for (int c = 0; c < 4; ++c) {
             mbar_init(&sm.it_full[c], kGathWarps);
