@@ -470,7 +470,12 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnOrder& ord,
     Unit u;
     for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
         if (u.t0 >= u.t1) continue;
-        const AttnProblem& P = ab.p[u.prob];
+        // the problem's fields in registers for the unit (a dynamically indexed
+        // kernel-parameter read per tile would miss the constant cache)
+        const uint8_t* const main_codes = ab.p[u.prob].cache.main_codes;
+        const uint8_t* const main_scales = ab.p[u.prob].cache.main_scales;
+        const uint8_t* const win8 = static_cast<const uint8_t*>(ab.p[u.prob].win);
+        const int PK = ab.p[u.prob].K;
         for (int t = u.t0; t < u.t1; ++t, ++it) {
             const int buf = it & 1;
             if (t == u.t0) {
@@ -489,8 +494,8 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnOrder& ord,
             uint32_t sc[4];
             if (kind == 1) {
                 const int64_t rw = sm.src_row[buf][r];
-                const uint8_t* codes = P.cache.main_codes + rw * MCB + 32 * hf;
-                const uint8_t* scl = P.cache.main_scales + rw * MSB + 4 * hf;
+                const uint8_t* codes = main_codes + rw * MCB + 32 * hf;
+                const uint8_t* scl = main_scales + rw * MSB + 4 * hf;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     cw[c][0] = __ldg(reinterpret_cast<const uint4*>(codes + 64 * c));
@@ -552,9 +557,8 @@ __device__ void role_gather(Smem& sm, const AttnBatch& ab, const AttnOrder& ord,
                         }
                     } else if (kind == 3) {
                         // E4M3 window row (slot t * 128 + r - K of the ring): 64 codes -> fp16 (exact)
-                        const int64_t rw = (int64_t)u.b * WIN + (t * kT + r - P.K);
-                        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(P.win) + rw * D +
-                                                                          128 * c + 64 * hf);
+                        const int64_t rw = (int64_t)u.b * WIN + (t * kT + r - PK);
+                        const uint4* src = reinterpret_cast<const uint4*>(win8 + rw * D + 128 * c + 64 * hf);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {  // 16 codes: chunks 2 q, 2 q + 1
                             const uint4 x = __ldg(src + (hf ? ((q + 2) & 3) : q));
