@@ -77,6 +77,7 @@ constexpr uint32_t kColO = 0;      // O^T: 4 blocks x 64 heads
 constexpr uint32_t kColS = 256;    // S^T: 64 heads
 constexpr uint32_t kColL = 320;    // per-lane partial row sums of P: 64 heads
 constexpr uint32_t kColM = 384;    // per-lane copy of the reference maxima: 64 heads
+constexpr uint32_t kColL2 = 448;   // the row sums' second buffer (a tile reads one, writes the other)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kGap2 = 8.0f * kLog2e;  // the reference maximum moves beyond e^8 (log2 units)
@@ -665,6 +666,7 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, const AttnOrder& ord
     const int H = ab.H;
     bool alive = true;
     uint32_t it = 0, ku = 0;
+    uint32_t lsel = 0;  // which row-sum buffer holds the sums so far
     Unit u;
     for (int k = 0; unit_at(ord, ab, splits, tps, k, u); ++k) {
         const bool partial = u.partial;
@@ -696,90 +698,96 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, const AttnOrder& ord
             if (lane == 0) mbar_arrive(&sm.lk_empty[buf]);
             alive = wait_bar_warp(sm, &sm.s_full, it & 1u) && alive;
             tc_fence_after();
-            // pass 1: does this item move a head's maximum?  (S^T and the lane's
-            // copy of the maxima from TMEM, a half at a time)
-            bool need = false;
-#pragma unroll 1  // unrolled, both halves' loads are hoisted together: 128 registers
-            for (int half = 0; half < 2; ++half) {
-                uint32_t sv[32], mv[32];
-                tmem_ld_x32_nowait(tl + kColS + 32 * half, sv);
-                tmem_ld_x32_nowait(tl + kColM + 32 * half, mv);
-                tmem_wait_ld2(sv, mv);
-#pragma unroll
-                for (int h = 0; h < 32; ++h)
-                    need |= fmaf(__uint_as_float(sv[h]), a2, -__uint_as_float(mv[h])) > kGap2;
-            }
-            if (named_bar_or(kBarSoft, 32 * kSoftWarps, (ok && need) || !alive)) {
-                // rare: the tile's maximum per head over the valid items
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float z[32];
-                    tmem_ld_32x32b_x32(tl + kColS + 32 * half, z);
-#pragma unroll
-                    for (int h = 0; h < 32; ++h) z[h] = ok ? z[h] * a2 : -INFINITY;
-                    sm.red[quad][32 * half + lane] = warp_reduce_scatter32<true>(z);
-                }
-                named_bar(kBarSoft, 32 * kSoftWarps);
-                bool resc = false;
-                if (st < kHp) {
-                    const float mt = fmaxf(fmaxf(sm.red[0][st], sm.red[1][st]), fmaxf(sm.red[2][st], sm.red[3][st]));
-                    const float mo = sm.mu2[st];
-                    float a = 1.0f;
-                    if (mt > mo + kGap2 || (mo == -INFINITY && mt != -INFINITY)) {
-                        a = (mo == -INFINITY) ? 0.0f : ex2(mo - mt);
-                        sm.mu2[st] = mt;
-                        resc = mo != -INFINITY;
-                    }
-                    sm.alpha[st] = a;
-                }
-                if (named_bar_or(kBarSoft, 32 * kSoftWarps, resc)) {
-                    // rescale the earlier tiles' O^T and row sums (the previous tile's O complete)
-                    alive = wait_bar_warp(sm, &sm.o_blk[3], (it - 1) & 1u) && alive;
-                    tc_fence_after();
+            const bool first = t == u.t0;
+            const uint32_t lcur = lsel ? kColL2 : kColL, lnext = lsel ? kColL : kColL2;
+            // p = exp2(scale 2^-k s - m) into P^T (fp16), and the lane's running row
+            // sums of the rounded p: read from lcur, written to lnext (so that a
+            // pass whose maxima turn out stale leaves them intact).  need: does
+            // this item move a head's maximum (by more than the gap)?
+            auto p_pass = [&](bool acc, bool& need) {
 #pragma unroll 1
-                    for (int c = 0; c < 10; ++c) {  // four O^T blocks, then the row sums, 32 columns at a time
-                        const uint32_t col = (c < 8 ? kColO + 32 * c : kColL + 32 * (c - 8));
-                        const int h0 = 32 * (c & 1);
-                        float o[32];
-                        tmem_ld_32x32b_x32(tl + col, o);
-#pragma unroll
-                        for (int h = 0; h < 32; ++h) o[h] *= sm.alpha[h0 + h];
-                        tmem_st_32x32b_x32(tl + col, o);
-                    }
-                }
-                // this lane's TMEM copy of the updated maxima
-#pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    float v[32];
+                    uint32_t sv[32], mv[32];
+                    tmem_ld_x32_nowait(tl + kColS + 32 * half, sv);
+                    tmem_ld_x32_nowait(tl + kColM + 32 * half, mv);
+                    tmem_wait_ld2(sv, mv);
+                    float y[32];
 #pragma unroll
-                    for (int h = 0; h < 32; ++h) v[h] = sm.mu2[32 * half + h];
-                    tmem_st_32x32b_x32(tl + kColM + 32 * half, v);
+                    for (int h = 0; h < 32; ++h) {
+                        y[h] = fmaf(__uint_as_float(sv[h]), a2, -__uint_as_float(mv[h]));
+                        need |= y[h] > kGap2;
+                    }
+                    store_p(sm.p, row, 4 * half, ok, y);
+                    if (acc) {
+                        float l[32];
+                        tmem_ld_32x32b_x32(tl + lcur + 32 * half, l);
+#pragma unroll
+                        for (int h = 0; h < 32; ++h) y[h] += l[h];
+                    }
+                    tmem_st_32x32b_x32(tl + lnext + 32 * half, y);
                 }
-            }
+            };
             // P^T is free once the previous tile's O has completed
             if (it > 0) alive = wait_bar_warp(sm, &sm.o_blk[3], (it - 1) & 1u) && alive;
-            // pass 2: p = exp2(scale 2^-k s - m) into P^T (fp16), and the lane's
-            // running row sums of the rounded p in TMEM
+            // a unit's first tile always sets the maxima; a later one is computed
+            // with the current maxima at once, and again only if one of them moves
+            // (one loop, so the pass is compiled once)
+            bool update = first;
+#pragma unroll 1
+            while (true) {
+                if (update) {
+                    // the tile's maximum per head over the valid items
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t sv[32], mv[32];
-                tmem_ld_x32_nowait(tl + kColS + 32 * half, sv);
-                tmem_ld_x32_nowait(tl + kColM + 32 * half, mv);
-                tmem_wait_ld2(sv, mv);
-                float y[32];
+                    for (int half = 0; half < 2; ++half) {
+                        float z[32];
+                        tmem_ld_32x32b_x32(tl + kColS + 32 * half, z);
 #pragma unroll
-                for (int h = 0; h < 32; ++h) y[h] = fmaf(__uint_as_float(sv[h]), a2, -__uint_as_float(mv[h]));
-                store_p(sm.p, row, 4 * half, ok, y);
-                if (t == u.t0) {
-                    tmem_st_32x32b_x32(tl + kColL + 32 * half, y);
-                } else {
-                    float l[32];
-                    tmem_ld_32x32b_x32(tl + kColL + 32 * half, l);
+                        for (int h = 0; h < 32; ++h) z[h] = ok ? z[h] * a2 : -INFINITY;
+                        sm.red[quad][32 * half + lane] = warp_reduce_scatter32<true>(z);
+                    }
+                    named_bar(kBarSoft, 32 * kSoftWarps);
+                    bool resc = false;
+                    if (st < kHp) {
+                        const float mt =
+                            fmaxf(fmaxf(sm.red[0][st], sm.red[1][st]), fmaxf(sm.red[2][st], sm.red[3][st]));
+                        const float mo = sm.mu2[st];
+                        float a = 1.0f;
+                        if (mt > mo + kGap2 || (mo == -INFINITY && mt != -INFINITY)) {
+                            a = (mo == -INFINITY) ? 0.0f : ex2(mo - mt);
+                            sm.mu2[st] = mt;
+                            resc = mo != -INFINITY;
+                        }
+                        sm.alpha[st] = a;
+                    }
+                    if (named_bar_or(kBarSoft, 32 * kSoftWarps, resc)) {
+                        // rescale the earlier tiles' O^T and row sums (the previous tile's O complete)
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c = 0; c < 10; ++c) {  // four O^T blocks, then the row sums, 32 columns at a time
+                            const uint32_t col = (c < 8 ? kColO + 32 * c : lcur + 32 * (c - 8));
+                            const int h0 = 32 * (c & 1);
+                            float o[32];
+                            tmem_ld_32x32b_x32(tl + col, o);
 #pragma unroll
-                    for (int h = 0; h < 32; ++h) l[h] += y[h];
-                    tmem_st_32x32b_x32(tl + kColL + 32 * half, l);
+                            for (int h = 0; h < 32; ++h) o[h] *= sm.alpha[h0 + h];
+                            tmem_st_32x32b_x32(tl + col, o);
+                        }
+                    }
+                    // this lane's TMEM copy of the updated maxima
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float v[32];
+#pragma unroll
+                        for (int h = 0; h < 32; ++h) v[h] = sm.mu2[32 * half + h];
+                        tmem_st_32x32b_x32(tl + kColM + 32 * half, v);
+                    }
                 }
+                bool need = false;
+                p_pass(!first, need);
+                if (update || !named_bar_or(kBarSoft, 32 * kSoftWarps, (ok && need) || !alive)) break;
+                update = true;
             }
+            lsel ^= 1u;
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
@@ -790,10 +798,11 @@ __device__ void role_softmax(Smem& sm, const AttnBatch& ab, const AttnOrder& ord
         alive = wait_bar_warp(sm, &sm.o_blk[3], (it - 1) & 1u) && alive;
         tc_fence_after();
         {
+            const uint32_t lfinal = lsel ? kColL2 : kColL;  // the buffer the unit's last tile wrote
             float l[32];
-            tmem_ld_32x32b_x32(tl + kColL, l);
+            tmem_ld_32x32b_x32(tl + lfinal, l);
             sm.red[quad][lane] = warp_reduce_scatter32<false>(l);
-            tmem_ld_32x32b_x32(tl + kColL + 32, l);
+            tmem_ld_32x32b_x32(tl + lfinal + 32, l);
             sm.red[quad][32 + lane] = warp_reduce_scatter32<false>(l);
         }
         named_bar(kBarSoft, 32 * kSoftWarps);
