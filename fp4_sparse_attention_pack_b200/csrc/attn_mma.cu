@@ -455,7 +455,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_h2_sat(uint32_t w) {
 
 // The eight gather warps write every slab pair of a tile together, pair after
 // pair, each as soon as the previous tile's O block that reads it has
-// completed, so a pair is ready a few hundred cycles after its block: thread
+// completed, so a pair is ready about a thousand cycles after its block: thread
 // (g, l) owns half h = l % 2 of row 16 g + l / 2 of every pair c, i.e. slab
 // 2 c + h of that row (64 channels: 32 code bytes, four scale bytes, one
 // 128-byte line of the image).  Odd lanes store their chunks four on, so that
