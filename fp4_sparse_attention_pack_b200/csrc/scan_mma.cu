@@ -416,7 +416,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if ((issued >> s) & 1u) (void)mbar_wait(&sm.full[s], (issued_par >> s) & 1u);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0, pass_no = 0;
+        // The pass loop keeps its per-pass work to the MMAs: the accumulator ring
+        // index and phase, the query descriptor and the scale column advance by
+        // constant steps, and the instruction descriptors are constants (this
+        // warp's issue rate, shared with busy epilogue warps, sets the pace).
+        uint32_t stage = 0, sphase = 0, bslot = 0, bphase = 0;
+        uint32_t acc = 0, aphase = 0;  // accumulator of the next pass, and its ring phase
+        constexpr uint32_t kIdesc2a = idesc_mxf4(kPass * kHeads, 0, 0), kIdesc2b = idesc_mxf4(kPass * kHeads, 2, 2);
+        constexpr uint32_t kIdesc1a = idesc_mxf4(kHeads, 0, 0), kIdesc1b = idesc_mxf4(kHeads, 2, 2);
         uint32_t* status = sb.p[0].cache.status;
         while (true) {
             if (!mbar_wait_warp(&sm.qfull[bslot], bphase)) {
@@ -432,6 +439,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (nprob == 0) break;
             status = D.status;
             const int passes = (nprob + kPass - 1) / kPass;
+            static_assert(kPass == 2, "a pass holds two problems, the last pass of an odd subset one");
+            const bool odd = (nprob & 1) != 0;
+            const uint64_t bdesc0 = smem_desc(sm.b[bslot], 16, 512, kLayoutSw64);
+            const uint32_t sfb0 = tbase + kColSfb + bslot * kMaxPasses * 4;
             // the item's query scales into TMEM (the columns' previous reader, the
             // item two back, has completed: its commit preceded this buffer's reload)
             tc_fence_after();
@@ -457,22 +468,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t sfa = tbase + kColSfa + 4 * stage;
                 tc_cp_32x128b_x4_w(sfa, smem_desc(sm.sfa_tc[stage], 16, 128, kLayoutNone));
                 const uint64_t adesc = smem_desc(sm.a[stage], 16, 512, kLayoutSw64);
-                for (int k = 0; k < passes; ++k, ++pass_no) {
-                    const uint32_t acc = pass_no % kAcc;
-                    if (!mbar_wait_warp(&sm.tempty[acc], ((pass_no / kAcc) & 1u) ^ 1u)) {
+                uint64_t bdesc = bdesc0;  // pass k: the queries of problems kPass k, kPass k + 1
+                uint32_t sfb = sfb0;      // and their scale columns
+#pragma unroll 1
+                for (int k = 0; k < passes; ++k) {
+                    if (!mbar_wait_warp(&sm.tempty[acc], aphase ^ 1u)) {
                         if (lane == 0) raise_abort(sm, status);
                         stop = true;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t n_rows = (uint32_t)min(kPass, nprob - kPass * k) * kHeads;
-                    const uint32_t sfb = tbase + kColSfb + (bslot * kMaxPasses + k) * 4;
+                    const bool one = odd && k + 1 == passes;  // an odd subset's last pass: one problem (N = 64)
                     const uint32_t d = tbase + kColAcc + 128 * acc;
-                    const uint64_t bdesc = smem_desc(sm.b[bslot] + k * kPass * kHeads * 64, 16, 512, kLayoutSw64);
                     // K = 0..63 (scale bytes 0, 1), then K = 64..127 (bytes 2, 3): +32 B start
-                    tc_mma_mxf4_w(d, adesc, bdesc, idesc_mxf4(n_rows, 0, 0), sfa, sfb, 0u);
-                    tc_mma_mxf4_w(d, adesc + 2, bdesc + 2, idesc_mxf4(n_rows, 2, 2), sfa, sfb, 1u);
+                    tc_mma_mxf4_w(d, adesc, bdesc, one ? kIdesc1a : kIdesc2a, sfa, sfb, 0u);
+                    tc_mma_mxf4_w(d, adesc + 2, bdesc + 2, one ? kIdesc1b : kIdesc2b, sfa, sfb, 1u);
                     tc_commit_w(&sm.tfull[acc]);
+                    bdesc += (uint64_t)((kPass * kHeads * 64) >> 4);
+                    sfb += 4;
+                    if (++acc == (uint32_t)kAcc) acc = 0, aphase ^= 1u;
                 }
                 if (stop) break;
                 tc_commit_w(&sm.empty[stage]);  // the stage is free once these MMAs complete
