@@ -20,8 +20,9 @@
 // MN-major A operand of O^T.  The reference maximum m_h only moves when a
 // tile's maximum exceeds it by more than 8 (so p <= e^8 fits fp16); the O
 // rescale that a move needs is rare, and a tile that moves no maximum needs no
-// cross-item reduction at all: every thread tests its own item against m_h and
-// one barrier ORs the tests.
+// cross-item reduction at all: every thread forms its item's P^T with the
+// current maxima while testing the item against them, one barrier ORs the
+// tests, and only a tile that moves a maximum is formed again.
 //
 // Persistent CTAs (one per SM, 480 threads) walk their units (problem,
 // sequence, split of tiles) tile by tile; warps specialise and hand work over
@@ -32,10 +33,11 @@
 //               row, or window slot) two tiles ahead, and prefetches the window
 //               rows and the next unit's query into L2;
 //   warps 2-5   softmax: thread = item row (TMEM lane), all 64 heads; P^T into
-//               shared memory; the per-lane partial row sums and a per-lane
-//               copy of the 64 reference maxima live in TMEM, so a tile's
-//               softmax reads no shared memory but its item's kind; at the end
-//               of a unit the O^T readout, normalised (or the split's partial);
+//               shared memory; the per-lane partial row sums (two buffers: a
+//               tile reads one and writes the other) and a per-lane copy of the
+//               64 reference maxima live in TMEM, so a tile's softmax reads no
+//               shared memory but its item's kind; at the end of a unit the
+//               O^T readout, normalised (or the split's partial);
 //   warps 6-13  gather: all eight write each slab pair of a tile (an O block's
 //               operand) together, pair after pair, as soon as the previous
 //               tile's O block that reads it has completed; each tile's entry
